@@ -1,0 +1,214 @@
+/*
+ * strata_moe.h -- C ABI of the B200 (sm_100a) mixture-of-experts expert layer.
+ *
+ * One MoE layer applied to a batch of T tokens (a prefill chunk, or a 1..4
+ * token decode / speculative-verify batch):
+ *
+ *   logits = x . W_r (+ bias)                 router
+ *   ids, w = top-k(logits), softmax over the k selected logits
+ *   rows grouped by expert (histogram -> exclusive scan -> stable scatter)
+ *   h      = SiLU(x . Wg_e) * (x . Wu_e)       grouped int4 GEMM, dequant fused
+ *   o      = h . Wd_e                           grouped int4 GEMM, dequant fused
+ *   y_t    = sum_j w_tj * o_(t,j)               weighted combine
+ *
+ * Sources.  The method is the MoE expert layer of the Strata local inference
+ * engine as described by public write-ups:
+ *   - each layer holds 512 experts and a token activates about 10; larger
+ *     prefill batches let more tokens reuse each expert: "两天移植，预填充提速8倍：
+ *     Strata引擎实测" (kongchang.com), section "Strata快在哪", MoE note;
+ *   - the per-layer router picks a subset of experts per token: penglei.dev
+ *     "Strata local MoE" post, section "原理一：把显存作为专家缓存";
+ *   - 4-bit group quantisation with per-group scales, group 32/64/128:
+ *     lqnn.cn static review section 3.1, yfxerp.com review section 3.1;
+ *   - dequantisation fused inside the matmul, never materialised: lqnn.cn
+ *     review sections 1.2 and 6.2, kongchang.com page section "Strata快在哪"
+ *     (MMQ note);
+ *   - activation fused with the FFN projection: yfxerp.com review section 5.1.
+ * The pages give no API, formula for the router, tie-break, activation or bit
+ * layout; the readings used here are stated at each declaration.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates or frees device memory; scratch space is the
+ *     caller's `ws` buffer of at least strata_moe_workspace_bytes(dims) bytes.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No call synchronises the host, so every call can be captured
+ *     in a CUDA graph.
+ *   - Arguments are validated on the host before any launch.  On error
+ *     nothing is launched and a status is returned; no exception crosses the
+ *     ABI and no kernel traps.
+ *   - Results are bit-identical from run to run (no floating-point atomics).
+ *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef STRATA_MOE_H
+#define STRATA_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define STRATA_API __attribute__((visibility("default")))
+#else
+#define STRATA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status of a call.  STRATA_ERR_DEVICE_CHECK is reported by
+ * strata_moe_device_status() when a kernel recorded a failed device-side
+ * check (an index out of range, or a bounded wait that ran out). */
+typedef enum {
+  STRATA_OK = 0,
+  STRATA_ERR_INVALID_ARG = 1,  /* null pointer, bad dims, misaligned pointer */
+  STRATA_ERR_UNSUPPORTED = 2,  /* valid shape this build does not implement */
+  STRATA_ERR_WORKSPACE = 3,    /* ws missing or smaller than required       */
+  STRATA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed       */
+  STRATA_ERR_DEVICE_CHECK = 5  /* a device-side check failed (see above)     */
+} strata_status_t;
+
+/* Layer dimensions.
+ *   T      tokens in the batch (T = 0 is a valid empty batch: nothing runs and
+ *          no pointer is read, except that strata_moe_permute zeroes counts
+ *          and offsets)
+ *   d      hidden size (reduction dim of gate/up, output dim of down)
+ *   E      number of experts
+ *   k      experts per token, 1 <= k <= E
+ *   n      expert intermediate size
+ *   group  int4 group size along K, for all three projections
+ * Supported: d, n multiples of 128; group in {32, 64, 128}; E <= 1024;
+ * k <= 32; T*k < 2^31.  Other positive shapes return STRATA_ERR_UNSUPPORTED. */
+typedef struct {
+  int32_t T, d, E, k, n, group;
+} strata_moe_dims_t;
+
+/* One group-quantised weight tensor for all E experts, logical W_e[K][N]
+ * (K = reduction dim), stored K-major per output feature:
+ *   q: [E][N][K/2] bytes.  Byte q[e][nn][kk/2] holds element kk in its low
+ *      nibble when kk is even and in its high nibble when kk is odd; nibbles
+ *      are two's-complement int4 in [-8, 7].
+ *   s: [E][N][K/group] fp16 scales.
+ * Element value: W_e[kk][nn] = q * s[e][nn][kk/group] (symmetric, no zero
+ * point).  gate/up: N = n, K = d.  down: N = d, K = n.  The pages describe
+ * grouped int4 with per-group scales (lqnn.cn review 3.1; yfxerp.com review
+ * 3.1) but no bit layout; this layout is the library's own. */
+typedef struct {
+  const uint8_t* q;
+  const uint16_t* s;
+} strata_q4_t;
+
+typedef enum {
+  STRATA_OP_GATE_UP_SWIGLU = 0, /* h = SiLU(a . Wg_e) * (a . Wu_e), a = gathered x */
+  STRATA_OP_DOWN = 1            /* o = a . Wd_e (times row_scale), a = h rows       */
+} strata_moe_op_t;
+
+/* A cudaStream_t without including CUDA headers. */
+typedef struct CUstream_st* strata_stream_t;
+
+/* Bytes of caller-provided scratch space that strata_moe_forward needs for
+ * `dims` (also enough for every other entry point).  Returns 0 for dims that
+ * no entry point accepts. */
+STRATA_API size_t strata_moe_workspace_bytes(strata_moe_dims_t dims);
+
+/* Static, NUL-terminated description of a status. */
+STRATA_API const char* strata_status_string(strata_status_t status);
+
+/* Router + top-k + softmax ("the router of each layer selects a subset of
+ * experts for every token": penglei.dev post, section "原理一").
+ *   x         [T][d] bf16, row-major
+ *   w_router  [d][E] bf16, row-major
+ *   bias      [E] fp32 or NULL; added to the logits before selection, and the
+ *             biased logits are the ones softmax weights are computed from
+ *   topk_ids  [T][k] int32 out: the k largest logits in descending order;
+ *             exactly equal logits go to the lower expert index
+ *   topk_w    [T][k] fp32 out: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ *             over the k selected logits (l_0 the largest)
+ *   logits_out [T][E] fp32 out or NULL: the fp32 logits selection used
+ *   ws/ws_bytes scratch (see strata_moe_workspace_bytes)
+ * Logits are accumulated in fp32 from bf16 products. */
+STRATA_API strata_status_t strata_moe_route(const uint16_t* x, const uint16_t* w_router,
+                                 const float* bias, strata_moe_dims_t dims,
+                                 int32_t* topk_ids, float* topk_w,
+                                 float* logits_out, void* ws, size_t ws_bytes,
+                                 strata_stream_t stream);
+
+/* Grouping of token slots by expert (tokens that share an expert are
+ * processed together: kongchang.com page, section "Strata快在哪", MoE note).
+ * Slot s = t*k + j is the j-th expert choice of token t.
+ *   topk_ids     [T][k] int32 in: expert of every slot, each in [0, E)
+ *   counts       [E] int32 out: number of slots routed to each expert
+ *   offsets      [E+1] int32 out: exclusive prefix sum of counts; offsets[E]=T*k
+ *   sorted_token [T*k] int32 out: row p -> token; rows of expert e are
+ *                offsets[e] .. offsets[e+1]-1 in increasing slot order
+ *   slot_row     [T*k] int32 out: slot s -> its row p
+ * The output is unique (a stable counting sort); ids outside [0, E) are
+ * clamped into range and reported through strata_moe_device_status(). */
+STRATA_API strata_status_t strata_moe_permute(const int32_t* topk_ids,
+                                   strata_moe_dims_t dims, int32_t* counts,
+                                   int32_t* offsets, int32_t* sorted_token,
+                                   int32_t* slot_row, void* ws, size_t ws_bytes,
+                                   strata_stream_t stream);
+
+/* Grouped expert projection with int4 dequantisation fused into the GEMM
+ * (dequantise inside the matmul: lqnn.cn review 1.2 / 6.2; expert matmul is
+ * the heaviest compute: kongchang.com page, "Strata快在哪"; activation fused
+ * with the projection: yfxerp.com review 5.1).
+ *   op = STRATA_OP_GATE_UP_SWIGLU:
+ *     a      [T][d] bf16 token rows (x); row p reads a[sorted_token[p]]
+ *     w0, w1 gate and up weights (N = n, K = d)
+ *     out    [T*k][n] bf16: out[p] = SiLU(a.Wg_e) * (a.Wu_e), e = expert of p
+ *     row_scale must be NULL
+ *   op = STRATA_OP_DOWN:
+ *     a      [T*k][n] bf16 rows in grouped order (the gate/up output)
+ *     sorted_token ignored (may be NULL); w0 = down weights (N = d, K = n);
+ *     w1 ignored
+ *     row_scale [T*k] fp32 or NULL: out[p] is multiplied by row_scale[p]
+ *     out    [T*k][d] bf16
+ *   offsets [E+1] int32: row ranges per expert, as from strata_moe_permute
+ * Products accumulate in fp32; dequantised weights are rounded to bf16. */
+STRATA_API strata_status_t strata_moe_expert_gemm_q4(
+    strata_moe_op_t op, const uint16_t* a, const int32_t* sorted_token,
+    const int32_t* offsets, strata_q4_t w0, strata_q4_t w1,
+    const float* row_scale, strata_moe_dims_t dims, uint16_t* out, void* ws,
+    size_t ws_bytes, strata_stream_t stream);
+
+/* Weighted combine back to token order:
+ *   y[t] = sum_{j=0..k-1} topk_w[t][j] * rows[slot_row[t*k+j]]
+ * summed in fp32 in the order j = 0..k-1 and rounded once to bf16.
+ *   rows     [T*k][d] bf16 (per-row expert outputs, grouped order)
+ *   topk_w   [T][k] fp32, or NULL when the rows are already weighted
+ *   slot_row [T*k] int32
+ *   y        [T][d] bf16 out */
+STRATA_API strata_status_t strata_moe_combine(const uint16_t* rows, const float* topk_w,
+                                   const int32_t* slot_row,
+                                   strata_moe_dims_t dims, uint16_t* y,
+                                   strata_stream_t stream);
+
+/* The whole layer: route -> permute -> gate/up -> down -> combine, stream
+ * ordered, all intermediates in `ws`.
+ *   x [T][d] bf16, w_router [d][E] bf16, bias [E] fp32 or NULL
+ *   gate, up (N = n, K = d), down (N = d, K = n): int4 weights as above
+ *   y [T][d] bf16 out
+ *   topk_ids_out [T][k] int32 / topk_w_out [T][k] fp32: optional copies of
+ *   the routes (NULL = not written) */
+STRATA_API strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router,
+                                   const float* bias, strata_q4_t gate,
+                                   strata_q4_t up, strata_q4_t down,
+                                   strata_moe_dims_t dims, uint16_t* y,
+                                   int32_t* topk_ids_out, float* topk_w_out,
+                                   void* ws, size_t ws_bytes,
+                                   strata_stream_t stream);
+
+/* Synchronises `stream`, then reports (and clears) the device-side check word
+ * of the current device: STRATA_OK, or STRATA_ERR_DEVICE_CHECK when a kernel
+ * since the last call recorded an out-of-range index or a bounded wait that
+ * timed out.  This is the one entry point that blocks the host. */
+STRATA_API strata_status_t strata_moe_device_status(strata_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STRATA_MOE_H */
