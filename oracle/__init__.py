@@ -55,9 +55,10 @@ def lib():
         L.oracle_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
         L.oracle_expert_ffn.argtypes = [vp] * 7 + [i64] * 4 + [vp, vp]
         L.oracle_moe_forward.argtypes = [vp] * 9 + [i64] * 6 + [vp, i64, vp, vp, vp, vp, vp, vp, vp]
-        L.oracle_combine.argtypes = [vp, vp, vp, i64, i64, i64, vp]
+        ci = ctypes.c_int
+        L.oracle_combine.argtypes = [vp, ci, vp, vp, i64, i64, i64, vp]
         L.oracle_gate_up_rows.argtypes = [vp, vp, i64, vp, vp, vp, vp, i64, i64, i64, vp]
-        L.oracle_down_rows.argtypes = [vp, vp, i64, vp, vp, vp, i64, i64, i64, vp]
+        L.oracle_down_rows.argtypes = [vp, ci, vp, i64, vp, vp, vp, i64, i64, i64, vp]
     return _lib
 
 
@@ -154,13 +155,14 @@ def moe_forward(inp, k: int, group: int, tokens=None, ids=None, w=None,
     return res
 
 
-def combine(rows, w, slot_row, T: int, k: int):
+def combine(rows, w, slot_row, T: int, k: int, rows_fp16: bool = False):
+    """rows: [S][d] bf16 bits (or fp16 bits with rows_fp16)."""
     rows = _c(rows, np.uint16)
     d = rows.shape[1]
     wv = None if w is None else _c(w, np.float64)
     sr = _c(slot_row, np.int32)
     y = np.empty((T, d), np.float64)
-    lib().oracle_combine(_p(rows), _p(wv), _p(sr), T, k, d, _p(y))
+    lib().oracle_combine(_p(rows), int(rows_fp16), _p(wv), _p(sr), T, k, d, _p(y))
     return y
 
 
@@ -176,7 +178,8 @@ def gate_up_rows(a, experts, inp, group: int):
     return out
 
 
-def down_rows(a, experts, inp, group: int, scale=None):
+def down_rows(a, experts, inp, group: int, scale=None, a_fp16: bool = False):
+    """a: [R][n] bf16 bits (or fp16 bits with a_fp16)."""
     a = _c(a, np.uint16)
     R, n = a.shape
     ex = _c(experts, np.int32)
@@ -184,6 +187,6 @@ def down_rows(a, experts, inp, group: int, scale=None):
     d = dq.shape[1]
     sc = None if scale is None else _c(scale, np.float32)
     out = np.empty((R, d), np.float64)
-    lib().oracle_down_rows(_p(a), _p(ex), R, _p(dq), _p(ds), _p(sc), d, n, group,
-                           _p(out))
+    lib().oracle_down_rows(_p(a), int(a_fp16), _p(ex), R, _p(dq), _p(ds), _p(sc), d, n,
+                           group, _p(out))
     return out

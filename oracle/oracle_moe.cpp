@@ -100,6 +100,9 @@ double dot_row(const double* v, const uint8_t* q, const uint16_t* s, int64_t K,
   return acc;
 }
 
+// Value of a 16-bit pattern stored as fp16 (is_f16 != 0) or bf16.
+double half_value(uint16_t v, int is_f16) { return is_f16 ? f16_value(v) : bf16_value(v); }
+
 }  // namespace
 
 extern "C" {
@@ -253,16 +256,16 @@ void oracle_moe_forward(const uint16_t* x, const uint16_t* w_router,
 }
 
 // Weighted combine of given per-slot rows (fp64): y[t] = sum_j w[t][j] *
-// rows[slot_row[t*k+j]].  rows are bf16 bits [S][d].
-void oracle_combine(const uint16_t* rows, const double* w, const int32_t* slot_row,
-                    int64_t T, int64_t k, int64_t d, double* y) {
+// rows[slot_row[t*k+j]].  rows are [S][d] fp16 (rows_f16 != 0) or bf16 bits.
+void oracle_combine(const uint16_t* rows, int rows_f16, const double* w,
+                    const int32_t* slot_row, int64_t T, int64_t k, int64_t d, double* y) {
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t) {
     for (int64_t i = 0; i < d; ++i) {
       double acc = 0.0;
       for (int64_t j = 0; j < k; ++j)
         acc += (w ? w[t * k + j] : 1.0) *
-               bf16_value(rows[static_cast<int64_t>(slot_row[t * k + j]) * d + i]);
+               half_value(rows[static_cast<int64_t>(slot_row[t * k + j]) * d + i], rows_f16);
       y[t * d + i] = acc;
     }
   }
@@ -292,9 +295,9 @@ void oracle_gate_up_rows(const uint16_t* a, const int32_t* experts, int64_t R,
   }
 }
 
-// The down projection alone on given bf16 rows: o[r][i] = a_r . Wd[e][i]
-// (times scale[r] when given).  a: [R][n] bf16 bits.  out: [R][d].
-void oracle_down_rows(const uint16_t* a, const int32_t* experts, int64_t R,
+// The down projection alone on given rows: o[r][i] = a_r . Wd[e][i] (times
+// scale[r] when given).  a: [R][n] fp16 (a_f16 != 0) or bf16 bits.  out: [R][d].
+void oracle_down_rows(const uint16_t* a, int a_f16, const int32_t* experts, int64_t R,
                       const uint8_t* down_q, const uint16_t* down_s,
                       const float* scale, int64_t d, int64_t n, int64_t G,
                       double* out) {
@@ -304,7 +307,7 @@ void oracle_down_rows(const uint16_t* a, const int32_t* experts, int64_t R,
     const uint8_t* dq = down_q + e * d * (n / 2);
     const uint16_t* ds = down_s + e * d * (n / G);
     std::vector<double> ar(n);
-    for (int64_t j = 0; j < n; ++j) ar[j] = bf16_value(a[r * n + j]);
+    for (int64_t j = 0; j < n; ++j) ar[j] = half_value(a[r * n + j], a_f16);
     for (int64_t i = 0; i < d; ++i) {
       const double o = dot_row(ar.data(), dq, ds, n, G, i);
       out[r * d + i] = scale ? o * static_cast<double>(scale[r]) : o;

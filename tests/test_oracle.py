@@ -277,6 +277,24 @@ def test_gate_up_and_down_rows_vs_dense():
         np.testing.assert_allclose(o[r], orr.numpy(), rtol=1e-10, atol=1e-12)
 
 
+def test_down_rows_and_combine_accept_fp16():
+    rng = np.random.default_rng(28)
+    inp = make_custom(T=4, d=128, E=2, k=1, n=64, group=32, seed=29)
+    h16 = (rng.standard_normal((5, 64)) * 3).astype(np.float16)
+    ex = np.array([1, 0, 1, 1, 0], np.int32)
+    o = oracle.down_rows(h16.view(np.uint16), ex, inp, 32, a_fp16=True)
+    for r in range(5):
+        Wd = dense_weights(inp["down_q"][ex[r]], inp["down_s"][ex[r]], 32)
+        ref = Wd @ torch.from_numpy(h16[r].astype(np.float64))
+        np.testing.assert_allclose(o[r], ref.numpy(), rtol=1e-12, atol=1e-12)
+    rows = (rng.standard_normal((6, 64)) * 10).astype(np.float16)
+    sr = np.array([5, 0, 3, 1, 2, 4], np.int32)
+    w = rng.uniform(0, 1, (3, 2))
+    y = oracle.combine(rows.view(np.uint16), w, sr, 3, 2, rows_fp16=True)
+    R = rows.astype(np.float64)[sr.reshape(3, 2)]
+    np.testing.assert_allclose(y, np.einsum("tk,tkd->td", w, R), rtol=1e-13, atol=1e-14)
+
+
 def test_combine_vs_einsum():
     rng = np.random.default_rng(25)
     T, k, d = 11, 3, 64
