@@ -40,6 +40,20 @@
  *   - Results are bit-identical from run to run (no floating-point atomics).
  *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
  *   - Device pointers must be 16-byte aligned.
+ *
+ * Numerics.  The layer input x and output y are bf16; the intermediates h and
+ * the per-row expert outputs are fp16, because fp16 carries the dequantised
+ * weights q*s to 2^-11 where bf16 would carry them to 2^-8, and bf16-rounded
+ * weights alone use up most of a 1.5e-2 * RMS error budget on these layers.
+ *   - router logits: fp32 accumulation of exact bf16 products;
+ *   - prefill batches (T > 8): tensor-core MMAs on fp16 operands -- x is
+ *     converted to fp16 (exact for |x| < 65504; larger values saturate to
+ *     infinity and are reported through strata_moe_device_status), each
+ *     weight is RNE_fp16(q * s), products accumulate in fp32;
+ *   - decode batches (T <= 8): the integer codes q enter the MMA exactly and
+ *     the fp16 group scale multiplies each group's fp32 partial sum;
+ *   - h = RNE_fp16(SiLU(g) * u), per-row outputs RNE_fp16(o);
+ *   - y = RNE_bf16(sum_j w_j * row_j), summed in fp32 in the order j = 0..k-1.
  */
 #ifndef STRATA_MOE_H
 #define STRATA_MOE_H
@@ -158,16 +172,18 @@ STRATA_API strata_status_t strata_moe_permute(const int32_t* topk_ids,
  *   op = STRATA_OP_GATE_UP_SWIGLU:
  *     a      [T][d] bf16 token rows (x); row p reads a[sorted_token[p]]
  *     w0, w1 gate and up weights (N = n, K = d)
- *     out    [T*k][n] bf16: out[p] = SiLU(a.Wg_e) * (a.Wu_e), e = expert of p
+ *     out    [T*k][n] fp16: out[p] = SiLU(a.Wg_e) * (a.Wu_e), e = expert of p
  *     row_scale must be NULL
  *   op = STRATA_OP_DOWN:
- *     a      [T*k][n] bf16 rows in grouped order (the gate/up output)
+ *     a      [T*k][n] fp16 rows in grouped order (the gate/up output)
  *     sorted_token ignored (may be NULL); w0 = down weights (N = d, K = n);
  *     w1 ignored
  *     row_scale [T*k] fp32 or NULL: out[p] is multiplied by row_scale[p]
- *     out    [T*k][d] bf16
- *   offsets [E+1] int32: row ranges per expert, as from strata_moe_permute
- * Products accumulate in fp32; dequantised weights are rounded to bf16. */
+ *     out    [T*k][d] fp16
+ *   offsets [E+1] int32: row ranges per expert, as from strata_moe_permute;
+ *     offsets that are not non-decreasing from 0 to T*k are reported through
+ *     strata_moe_device_status() and nothing is computed
+ * Products accumulate in fp32 (see Numerics above). */
 STRATA_API strata_status_t strata_moe_expert_gemm_q4(
     strata_moe_op_t op, const uint16_t* a, const int32_t* sorted_token,
     const int32_t* offsets, strata_q4_t w0, strata_q4_t w1,
@@ -177,7 +193,7 @@ STRATA_API strata_status_t strata_moe_expert_gemm_q4(
 /* Weighted combine back to token order:
  *   y[t] = sum_{j=0..k-1} topk_w[t][j] * rows[slot_row[t*k+j]]
  * summed in fp32 in the order j = 0..k-1 and rounded once to bf16.
- *   rows     [T*k][d] bf16 (per-row expert outputs, grouped order)
+ *   rows     [T*k][d] fp16 (per-row expert outputs, grouped order)
  *   topk_w   [T][k] fp32, or NULL when the rows are already weighted
  *   slot_row [T*k] int32
  *   y        [T][d] bf16 out */

@@ -119,14 +119,20 @@ Schedule schedule_at(uint8_t* ws, const SchedRegions& r) {
   s.n_active = reinterpret_cast<int32_t*>(ws + r.n_active.off);
   return s;
 }
+// fp16 copy of x used by the tensor-core gate/up path (batches above the
+// streaming threshold).
+size_t x16_bytes(const strata_moe_dims_t& d) {
+  return d.T > kStreamMaxTokens ? (size_t)d.T * d.d * 2 : 0;
+}
 size_t gemm_scratch(const strata_moe_dims_t& d) {
   Layout L;
   add_schedule(L, d);
+  L.add(x16_bytes(d));
   return L.total;
 }
 
 struct ForwardLayout {
-  Region ids, w, partial, counts, offsets, sorted_token, slot_row, hist, h, rows;
+  Region ids, w, partial, counts, offsets, sorted_token, slot_row, hist, x16, h, rows;
   SchedRegions sched;
   size_t total;
 };
@@ -143,6 +149,7 @@ ForwardLayout forward_layout(const strata_moe_dims_t& d) {
   f.slot_row = L.add(S * sizeof(int32_t));
   f.hist = L.add(permute_scratch(d));
   f.sched = add_schedule(L, d);
+  f.x16 = L.add(x16_bytes(d));
   f.h = L.add(S * (size_t)d.n * 2);
   f.rows = L.add(S * (size_t)d.d * 2);
   f.total = L.total;
@@ -168,10 +175,11 @@ strata_status_t do_route(const uint16_t* x, const uint16_t* w_router, const floa
 strata_status_t do_gemm(int op, const uint16_t* a, const int32_t* sorted_token,
                         const int32_t* offsets, strata_q4_t w0, strata_q4_t w1,
                         const float* row_scale, const strata_moe_dims_t& d, uint16_t* out,
-                        const Schedule& sch, unsigned* err, cudaStream_t s) {
+                        const Schedule& sch, uint16_t* x16, unsigned* err, cudaStream_t s) {
   GemmProblem p;
   p.op = op;
   p.a = a;
+  p.a16 = x16;
   p.sorted_token = sorted_token;
   p.offsets = offsets;
   p.q0 = w0.q;
@@ -278,11 +286,13 @@ strata_status_t strata_moe_expert_gemm_q4(strata_moe_op_t op, const uint16_t* a,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Layout L;
   const SchedRegions r = add_schedule(L, dims);
+  const Region x16 = L.add(x16_bytes(dims));
   const Schedule sch = schedule_at(static_cast<uint8_t*>(ws), r);
   if (launch_schedule(offsets, dims.E, dims.T * dims.k, sch, err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
   return do_gemm(op == STRATA_OP_GATE_UP_SWIGLU ? 0 : 1, a, sorted_token, offsets, w0, w1,
-                 row_scale, dims, out, sch, err, s);
+                 row_scale, dims, out, sch,
+                 reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + x16.off), err, s);
 }
 
 strata_status_t strata_moe_combine(const uint16_t* rows, const float* topk_w,
@@ -336,10 +346,11 @@ strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router, 
     return STRATA_ERR_CUDA;
   if (launch_schedule(offsets, dims.E, dims.T * dims.k, sch, err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
-  st = do_gemm(0, x, sorted_token, offsets, gate, up, nullptr, dims, h, sch, err, s);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(at(f.x16));
+  st = do_gemm(0, x, sorted_token, offsets, gate, up, nullptr, dims, h, sch, x16, err, s);
   if (st != STRATA_OK) return st;
   const strata_q4_t none = {nullptr, nullptr};
-  st = do_gemm(1, h, nullptr, offsets, down, none, nullptr, dims, rows, sch, err, s);
+  st = do_gemm(1, h, nullptr, offsets, down, none, nullptr, dims, rows, sch, x16, err, s);
   if (st != STRATA_OK) return st;
   return cuda_status(launch_combine_checked(rows, w, slot_row, dims.T, dims.k, dims.d, y, err, s));
 }

@@ -1,7 +1,7 @@
 // combine.cu -- weighted scatter-combine of the per-row expert outputs back
 // to token order:  y[t] = sum_{j<k} w[t][j] * rows[slot_row[t*k+j]].
 //
-// Memory bound (reads T*k rows of d bf16, writes T rows).  One CTA of 128
+// Memory bound (reads T*k fp16 rows of d values, writes T bf16 rows).  One CTA of 128
 // threads per token row; each thread owns 8 consecutive features and reads
 // them with 16-byte loads from all k rows before accumulating in fp32 in the
 // fixed order j = 0..k-1 (deterministic, no atomics), then rounds once.
@@ -43,8 +43,8 @@ __global__ void __launch_bounds__(128)
         const uint32_t p[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = fmaf(wj, bf16_lo(p[i]), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(wj, bf16_hi(p[i]), acc[2 * i + 1]);
+          acc[2 * i] = fmaf(wj, f16_lo(p[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wj, f16_hi(p[i]), acc[2 * i + 1]);
         }
       }
     }
@@ -54,8 +54,8 @@ __global__ void __launch_bounds__(128)
       const uint32_t p[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(wj, bf16_lo(p[i]), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(wj, bf16_hi(p[i]), acc[2 * i + 1]);
+        acc[2 * i] = fmaf(wj, f16_lo(p[i]), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj, f16_hi(p[i]), acc[2 * i + 1]);
       }
     }
     uint4 o;

@@ -18,6 +18,7 @@ namespace strata {
 enum : unsigned {
   kErrIndex = 1u,        // an index read from an input was out of range
   kErrTimeout = 2u,      // a bounded wait gave up
+  kErrRange = 4u,        // a value outside the fp16 range met an fp16 operand
 };
 
 // A wait that has not completed after this long is abandoned (the kernel
@@ -143,8 +144,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (fp16 or bf16 inputs as
+// the instruction descriptor says), fp32 accumulate.
+__device__ __forceinline__ void mma_f16kind_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -207,13 +209,16 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t 
          ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
-// Instruction descriptor for kind::f16: bf16 A and B, fp32 D, M x N tile.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
-//   15 A major (0 = K), 16 B major (0 = K, 1 = MN), 17-22 N >> 3, 24-28 M >> 4.
-__device__ __forceinline__ uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((N >> 3) << 17) |
-         ((M >> 4) << 24);
+// Instruction descriptor for kind::f16 with fp32 D and an M x N tile.
+//   bits 4-5 D format (1 = f32), 7-9 A format and 10-12 B format (0 = f16,
+//   1 = bf16), 15 A major (0 = K), 16 B major (0 = K, 1 = MN),
+//   17-22 N >> 3, 24-28 M >> 4.
+__device__ __forceinline__ uint32_t idesc_f32acc(uint32_t M, uint32_t N, uint32_t ab_format,
+                                                 uint32_t b_mn_major) {
+  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_mn_major << 16) |
+         ((N >> 3) << 17) | ((M >> 4) << 24);
 }
+constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
 
 // Offset of 16-byte chunk `c` (0..7) of row `r` in a K-major 128B-swizzled
 // tile whose rows are 128 bytes.
@@ -231,6 +236,16 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+__device__ __forceinline__ uint16_t f16_bits(float v) {
+  return __half_as_ushort(__float2half_rn(v));
 }
 
 }  // namespace strata

@@ -1,5 +1,7 @@
 // gemm_stream.cu -- expert projections for decode / speculative-verify
 // batches (T <= 8 tokens, so every expert sees at most a few rows).
+// Gate/up multiplies bf16 x by the exact integer codes as bf16; down
+// multiplies the fp16 h rows by the codes as fp16; outputs are fp16.
 //
 // Decoding gives no large batch to hide behind; every token needs its experts'
 // weights read again (kongchang.com "两天移植，预填充提速8倍：Strata引擎实测",
@@ -27,22 +29,37 @@ constexpr int THREADS = WARPS * 32;
 constexpr int UNROLL = 4;          // 64-K blocks whose loads are in flight together
 }  // namespace st
 
-// bf16 pair (136 + q_i, 136 + q_{i+4}) from nibbles i and i+4 of w, then the
-// exact subtraction of 136.
+// Exact integer pair (q_i, q_{i+4}) from nibbles i and i+4 of w, as bf16x2
+// (F16 = false: 136 + q in the mantissa of 128.0) or fp16x2 (F16 = true:
+// 1032 + q in the mantissa of 1024.0), then the exact subtraction.
+template <bool F16>
 __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
-  const uint32_t v = (((w >> (4 * i)) ^ 0x43084308u) & 0x000F000Fu) | 0x43004300u;
   uint32_t q;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
+  if (F16) {
+    const uint32_t v = (((w >> (4 * i)) ^ 0x64086408u) & 0x000F000Fu) | 0x64006400u;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
+  } else {
+    const uint32_t v = (((w >> (4 * i)) ^ 0x43084308u) & 0x000F000Fu) | 0x43004300u;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
+  }
   return q;
 }
 
+template <bool F16>
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  if (F16)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 struct StreamArgs {
@@ -62,12 +79,15 @@ struct StreamArgs {
 
 // One 32-wide half-block for one weight matrix: two MMAs on 8 nibbles per
 // row (rows g and g+8), result scaled into acc.
+template <bool F16>
 __device__ __forceinline__ void half_block(float (&acc)[4], uint32_t wg, uint32_t wg8,
                                            float sg, float sg8, uint32_t b00, uint32_t b01,
                                            uint32_t b10, uint32_t b11) {
   float c[4] = {0.f, 0.f, 0.f, 0.f};
-  mma16816(c, nib_pair(wg, 0), nib_pair(wg8, 0), nib_pair(wg, 1), nib_pair(wg8, 1), b00, b01);
-  mma16816(c, nib_pair(wg, 2), nib_pair(wg8, 2), nib_pair(wg, 3), nib_pair(wg8, 3), b10, b11);
+  mma16816<F16>(c, nib_pair<F16>(wg, 0), nib_pair<F16>(wg8, 0), nib_pair<F16>(wg, 1),
+                nib_pair<F16>(wg8, 1), b00, b01);
+  mma16816<F16>(c, nib_pair<F16>(wg, 2), nib_pair<F16>(wg8, 2), nib_pair<F16>(wg, 3),
+                nib_pair<F16>(wg8, 3), b10, b11);
   acc[0] = fmaf(sg, c[0], acc[0]);
   acc[1] = fmaf(sg, c[1], acc[1]);
   acc[2] = fmaf(sg8, c[2], acc[2]);
@@ -152,10 +172,10 @@ __global__ void __launch_bounds__(st::THREADS)
               const uint32_t b01 = __byte_perm(x.x, x.z, 0x7632);   // (1, 5)
               const uint32_t b10 = __byte_perm(x.y, x.w, 0x5410);   // (2, 6)
               const uint32_t b11 = __byte_perm(x.y, x.w, 0x7632);   // (3, 7)
-              half_block(acc0, wa[j][h][0], wa[j][h][1], __half2float(__ushort_as_half(__ldg(sg0 + grp))),
+              half_block<NMAT == 1>(acc0, wa[j][h][0], wa[j][h][1], __half2float(__ushort_as_half(__ldg(sg0 + grp))),
                          __half2float(__ushort_as_half(__ldg(sg0b + grp))), b00, b01, b10, b11);
               if (NMAT == 2)
-                half_block(acc1, wb[j][h][0], wb[j][h][1],
+                half_block<false>(acc1, wb[j][h][0], wb[j][h][1],
                            __half2float(__ushort_as_half(__ldg(sg1 + grp))),
                            __half2float(__ushort_as_half(__ldg(sg1b + grp))), b00, b01, b10, b11);
             }
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(st::THREADS)
             v = acc0[i];
             if (args.row_scale) v *= args.row_scale[p_begin + col];
           }
-          args.out[(size_t)(p_begin + col) * N + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          args.out[(size_t)(p_begin + col) * N + feat] = f16_bits(v);
         }
       }
     }

@@ -21,10 +21,14 @@
 //   warps 2-5  dequantise packed -> bf16 into the 128-byte-swizzled A tile
 //              (thread = weight row), then run the epilogue of the unit from
 //              TMEM (SwiGLU for gate/up, row scale for down)
-// Dequantisation: q in [-8, 7] becomes the bf16 value 136 + q by placing the
-// nibble (sign bit flipped) in the mantissa of 128.0, one fma subtracts 136
-// exactly, and one bf16 multiply applies the group scale (the fp16 scale is
-// rounded to bf16 first), so each weight is RNE_bf16(q * bf16(s)).
+// Operands are fp16 (kind::f16 with f16 A and B): the gathered token rows are
+// an fp16 copy of x (exact for |x| < 65504; made once per call), h is kept in
+// fp16, and each dequantised weight is RNE_fp16(q * s) -- fp16 holds q * s to
+// 2^-11, where bf16 weights (2^-8) would cost the layer most of its error
+// budget.  Dequantisation: q in [-8, 7] becomes the fp16 value 1032 + q by
+// placing the nibble (sign bit flipped) in the mantissa of 1024.0, one fma
+// subtracts 1032 exactly, and one fp16 multiply by the fp16 group scale
+// rounds once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -69,7 +73,7 @@ struct TcArgs {
   unsigned* err;
 };
 
-// 8 int4 (natural order: nibble i = element i) -> 8 bf16 = RNE(q_i * sc).
+// 8 int4 (natural order: nibble i = element i) -> 8 fp16 = RNE(q_i * s).
 __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t sc2) {
   const uint32_t w4 = w >> 4;
   uint32_t r[4];
@@ -78,21 +82,40 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t sc2) {
     // byte i of w (element 2i in its low nibble) to the low half, byte i of
     // w >> 4 (element 2i+1 in its low nibble) to the high half
     const uint32_t t = __byte_perm(w, w4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
-    // bf16 pair 128 + (nibble ^ 8) = 136 + q
-    const uint32_t v = ((t ^ 0x43084308u) & 0x000F000Fu) | 0x43004300u;
+    // fp16 pair 1024 + (nibble ^ 8) = 1032 + q
+    const uint32_t v = ((t ^ 0x64086408u) & 0x000F000Fu) | 0x64006400u;
     uint32_t qv, o;
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(qv) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o) : "r"(qv), "r"(sc2));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(qv) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o) : "r"(qv), "r"(sc2));
     r[i] = o;
   }
   return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-__device__ __forceinline__ uint32_t scale_bf16x2(uint16_t s_f16) {
-  const float f = __half2float(__ushort_as_half(s_f16));
-  const __nv_bfloat16 b = __float2bfloat16_rn(f);
-  const uint32_t u = __bfloat16_as_ushort(b);
-  return u | (u << 16);
+__device__ __forceinline__ uint32_t scale_f16x2(uint16_t s_f16) {
+  return (uint32_t)s_f16 | ((uint32_t)s_f16 << 16);
+}
+
+// fp16 copy of bf16 rows (the gathered B operand of the gate/up GEMM).
+// Values beyond the fp16 range become +-inf and are reported as kErrRange.
+__global__ void __launch_bounds__(256)
+    bf16_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n8,
+                       unsigned* err) {
+  bool over = false;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = src[i];
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = bf16_lo(in[j]), hi = bf16_hi(in[j]);
+      over |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+      out[j] = (uint32_t)f16_bits(lo) | ((uint32_t)f16_bits(hi) << 16);
+    }
+    dst[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (over) atomicOr(err, kErrRange);
 }
 
 template <int NMAT>
@@ -209,7 +232,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int p0 = args.offsets[e] + te.y * NT;
         const int cnt = min(NT, args.offsets[e + 1] - p0);
         const int nrows = (cnt + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(BM, nrows, 0);
+        const uint32_t idesc = idesc_f32acc(BM, nrows, kFmtF16, 0);
         if (i > 0) {
           if (!mbar_wait(acc_empty, (i - 1) & 1, abort_flag, args.err)) break;
           tc_fence_after();
@@ -232,7 +255,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             for (int m = 0; m < NMAT; ++m) {
               const uint64_t ad =
                   desc_kmajor_sw128(smem_addr(sA + (s * NMAT + m) * A_BYTES) + ks * 32);
-              mma_bf16_ss(tmem + m * NT, ad, bd, idesc, (kb | ks) != 0);
+              mma_f16kind_ss(tmem + m * NT, ad, bd, idesc, (kb | ks) != 0);
             }
           }
           mma_commit(&empty[s]);
@@ -265,11 +288,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int g0 = (kb * BK) / G;
         const int g1 = (kb * BK + BK / 2) / G;
         uint32_t sc[NMAT][2];
-        sc[0][0] = scale_bf16x2(__ldg(srow0 + g0));
-        sc[0][1] = g1 == g0 ? sc[0][0] : scale_bf16x2(__ldg(srow0 + g1));
+        sc[0][0] = scale_f16x2(__ldg(srow0 + g0));
+        sc[0][1] = scale_f16x2(__ldg(srow0 + g1));
         if (NMAT == 2) {
-          sc[NMAT - 1][0] = scale_bf16x2(__ldg(srow1 + g0));
-          sc[NMAT - 1][1] = g1 == g0 ? sc[NMAT - 1][0] : scale_bf16x2(__ldg(srow1 + g1));
+          sc[NMAT - 1][0] = scale_f16x2(__ldg(srow1 + g0));
+          sc[NMAT - 1][1] = scale_f16x2(__ldg(srow1 + g1));
         }
         if (!mbar_wait(&raw_full[s], ph, abort_flag, args.err)) {
           stop = true;
@@ -313,7 +336,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
               const float gv = __uint_as_float(acc0[j]);
               const float uv = __uint_as_float(acc1[j]);
               const float h = gv / (1.0f + __expf(-gv)) * uv;
-              args.out[(size_t)(p0 + p) * N + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+              args.out[(size_t)(p0 + p) * N + feat] = f16_bits(h);
             }
           }
         } else {
@@ -324,7 +347,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             if (p < cnt) {
               float v = __uint_as_float(acc0[j]);
               if (args.row_scale) v *= args.row_scale[p0 + p];
-              args.out[(size_t)(p0 + p) * N + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+              args.out[(size_t)(p0 + p) * N + feat] = f16_bits(v);
             }
           }
         }
@@ -359,12 +382,10 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                      tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  static bool configured = false;
-  if (!configured) {
+  {
     cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<NMAT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   if (g_num_sms == 0) {
     int dev = 0;
@@ -372,8 +393,16 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
     cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (g_num_sms <= 0) g_num_sms = 148;
   }
+  if (p.op == 0) {
+    // the gate/up B operand is the fp16 copy of x
+    const size_t n8 = (size_t)p.T * p.K / 8;
+    int blocks = (int)((n8 + 255) / 256);
+    if (blocks > 8 * g_num_sms) blocks = 8 * g_num_sms;
+    bf16_to_f16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(p.a),
+                                              reinterpret_cast<uint4*>(p.a16), n8, p.err);
+  }
   TcArgs a;
-  a.a = p.a;
+  a.a = p.op == 0 ? p.a16 : p.a;
   a.sorted_token = p.sorted_token;
   a.offsets = p.offsets;
   a.tile_table = sch.tile_table;

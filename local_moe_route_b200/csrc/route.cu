@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, 1);
+      const uint32_t idesc = idesc_f32acc(BM, BN, kFmtBF16, 1);
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         if (!mbar_wait(&full[s], (kb / STAGES) & 1, abort_flag, err)) break;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
         for (int ks = 0; ks < BK / 16; ++ks) {
           const uint64_t ad = desc_kmajor_sw128(a0 + ks * 32);
           const uint64_t bd = desc_mnmajor_sw128(b0 + ks * 16 * 128, B_BYTES / 2);
-          mma_bf16_ss(tmem, ad, bd, idesc, (kb | ks) != 0);
+          mma_f16kind_ss(tmem, ad, bd, idesc, (kb | ks) != 0);
         }
         mma_commit(&empty[s]);
       }
@@ -150,12 +150,10 @@ cudaError_t launch_router_logits_tc(const uint16_t* x, const uint16_t* w_router,
                      rt::BK, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  static bool configured = false;   // attribute is per function, idempotent
-  if (!configured) {
+  {
     cudaError_t e = cudaFuncSetAttribute(router_logits_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, rt::SMEM);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   dim3 grid((T + rt::BM - 1) / rt::BM, E / rt::BN);
   router_logits_tc_kernel<<<grid, rt::THREADS, rt::SMEM, s>>>(mx, mw, T, d, E, logits, err);

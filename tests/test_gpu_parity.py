@@ -1,18 +1,24 @@
 """GPU parity: every step of the layer, through the C ABI, against the fp64
-oracle on the same seeded inputs.
+oracle.  Both sides always receive the same seeded inputs: intermediates that
+a step consumes (routes, grouped rows, h, per-row outputs) are drawn by the
+test or derived by the oracle, never taken from the GPU.
 
-Bars (integer work bit-exact, floating point within the output gate):
-  * router logits: |gpu - oracle| <= 1e-4 * RMS(logits) (fp32 accumulation);
-  * expert ids: identical to the oracle's top-k run on the GPU's own fp32
-    logits, and identical to the oracle's fp64 routing except where the
-    oracle's own logits are within 1e-4*RMS of a tie (none for these seeds);
-  * routing weights: within 1e-6 of the oracle's softmax on the GPU logits;
-  * counts, offsets, sorted_token, slot_row: bit-exact;
-  * bf16 outputs (h, per-row outputs, y): max |gpu - oracle| <= 1.5e-2 *
-    RMS(oracle), the layer's output gate.
+Bars:
+  * expert ids, counts, offsets, sorted_token, slot_row: bit-exact.  With
+    integer-valued router inputs the fp32 and fp64 logits coincide, so the
+    top-k (including its lowest-index tie-break) must match exactly.  With
+    real-valued inputs a route may differ only where the oracle's logits lie
+    within the fp32 accumulation error of a tie (several answers are correct
+    there; none occur for most seeds and the count is reported);
+  * router logits within 1e-4 * RMS of the oracle; routing weights within
+    1e-5 where the routes agree;
+  * floating-point outputs: max(|gpu - oracle| - half_ulp(oracle)) <= 1.5e-2
+    * RMS(oracle), i.e. the layer's 1.5e-2 * RMS gate on top of the output
+    format's own correct rounding (bf16 y: half an ulp is 2^-8 relative, and
+    these outputs peak near 6 RMS, so even an exactly computed y rounded to
+    bf16 can miss a gate that does not allow for it).
 Large workloads are checked on seeded samples of rows/tokens (the oracle is
-per token, so a sample is exact), in the launch configuration the benchmark
-uses.
+per token, so a sample is exact), in the launch configuration of the bench.
 """
 
 import gc
@@ -23,9 +29,9 @@ import torch
 
 import local_moe_route_b200 as sm
 import oracle
-from gpu_helpers import (Layer, assert_device_ok, bf16_host, bf16_to_f64, gate_error,
-                         near_tie_tokens, rms)
-from moe_inputs import WORKLOADS, chunk_sizes
+from gpu_helpers import (Layer, assert_device_ok, bf16_host, bf16_to_f64, f16_host, f16_to_f64,
+                         gate_error, raw_error, rms)
+from moe_inputs import WORKLOADS, bf16_bits, chunk_sizes, make_custom
 
 pytestmark = pytest.mark.gpu
 
@@ -58,14 +64,21 @@ def sample(n, m, seed):
     return np.sort(np.random.default_rng(seed).choice(n, m, replace=False))
 
 
-def ids_agree(ids_gpu, logits_ref, k):
-    """GPU ids equal the oracle's fp64 routing except on near-tie tokens."""
-    ids_ref, _ = oracle.topk_softmax(logits_ref, k)
+def oracle_routes(L, tokens=None):
+    x = L.inp["x"] if tokens is None else L.inp["x"][tokens]
+    lg = oracle.router_logits(x, L.inp["w_router"], L.inp.get("bias"))
+    ids, w = oracle.topk_softmax(lg, L.dims["k"])
+    return lg, ids, w
+
+
+def routes_agree(ids_gpu, lg_ref, k, tol):
+    """GPU routes equal the oracle's except where a tie lies within `tol`
+    (the bound on the GPU's logit error) among the first k+1 sorted logits.
+    Returns (near-tie tokens, mismatching tokens)."""
+    ids_ref, _ = oracle.topk_softmax(lg_ref, k)
     mism = np.any(ids_gpu != ids_ref, axis=1)
-    # a near tie anywhere among the first k+1 sorted logits can reorder picks
-    srt = -np.sort(-logits_ref, axis=1)[:, :k + 1]
-    gaps = -np.diff(srt, axis=1)
-    ties = np.any(gaps < 1e-4 * rms(logits_ref), axis=1)
+    srt = -np.sort(-lg_ref, axis=1)[:, :k + 1]
+    ties = np.any(-np.diff(srt, axis=1) <= 2 * tol, axis=1)
     assert not np.any(mism & ~ties), np.nonzero(mism & ~ties)[0][:10]
     return int(ties.sum()), int(mism.sum())
 
@@ -77,32 +90,52 @@ def test_route(name, dev):
     wl = WORKLOADS[name]
     ids, w, logits = L.route()
     assert_device_ok()
-    lg = logits.cpu().numpy().astype(np.float64)
     rows = sample(wl.T, 1024, 7)
-    ref = oracle.router_logits(L.inp["x"][rows], L.inp["w_router"], L.inp.get("bias"))
-    assert np.max(np.abs(lg[rows] - ref)) <= 1e-4 * rms(ref) + 1e-6
-    # the same decisions as the oracle's top-k on the GPU's own fp32 logits
-    ids_o, w_o = oracle.topk_softmax(lg, wl.k)
-    assert np.array_equal(ids.cpu().numpy(), ids_o)
-    assert np.max(np.abs(w.cpu().numpy() - w_o)) <= 1e-6
-    ntie, nmis = ids_agree(ids.cpu().numpy()[rows], ref, wl.k)
-    assert nmis == 0, (ntie, nmis)
+    lg_ref, ids_ref, w_ref = oracle_routes(L, rows)
+    lg = logits.cpu().numpy().astype(np.float64)[rows]
+    err = np.max(np.abs(lg - lg_ref))
+    assert err <= 1e-4 * rms(lg_ref) + 1e-6, err
+    ids_g = ids.cpu().numpy()[rows]
+    ntie, nmis = routes_agree(ids_g, lg_ref, wl.k, err)
+    same = np.all(ids_g == ids_ref, axis=1)
+    assert np.max(np.abs(w.cpu().numpy()[rows][same] - w_ref[same])) <= 1e-5
+    print(f"{name}: logit err {err:.2e}, near-tie tokens {ntie}, differing routes {nmis}")
+
+
+@pytest.mark.parametrize("T,E,k", [(300, 128, 8), (5, 128, 8), (70, 32, 32), (1, 16, 3)])
+def test_route_integer_logits_exact(T, E, k, dev):
+    """x and W_r hold small integers (times 2^-4), so every partial sum is exact
+    in fp32 and the GPU's logits equal the oracle's bit for bit.  Integer
+    logits tie often: the lowest-index rule decides many slots."""
+    rng = np.random.default_rng(T + E)
+    d = 256
+    L = Layer.custom(dev, T=T, d=d, E=E, k=k, n=128, group=64, seed=60)
+    L.inp["x"] = bf16_bits(rng.integers(-2, 3, (T, d)).astype(np.float32))
+    L.inp["w_router"] = bf16_bits(rng.integers(-2, 3, (d, E)).astype(np.float32) / 16)
+    L.x = torch.from_numpy(L.inp["x"]).to(dev).view(torch.bfloat16)
+    L.w_router = torch.from_numpy(L.inp["w_router"]).to(dev).view(torch.bfloat16)
+    ids, w, logits = L.route()
+    assert_device_ok()
+    lg_ref, ids_ref, w_ref = oracle_routes(L)
+    assert np.array_equal(logits.cpu().numpy().astype(np.float64), lg_ref)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.max(np.abs(w.cpu().numpy() - w_ref)) <= 1e-6
+    if T * k >= 40:
+        srt = -np.sort(-lg_ref, axis=1)[:, :k + 1]
+        assert np.any(np.diff(srt, axis=1) == 0), "the case should contain exact ties"
 
 
 def test_route_skewed_chunk(dev):
     L = layer_for("skewed", dev)
     wl = WORKLOADS["skewed"]
-    x = L.x[:6144]
-    ids, w, logits = L.route(x)
-    lg = logits.cpu().numpy().astype(np.float64)
+    ids, w, logits = L.route(L.x[:6144])
     rows = sample(6144, 512, 8)
-    ref = oracle.router_logits(L.inp["x"][rows], L.inp["w_router"], L.inp["bias"])
-    assert np.max(np.abs(lg[rows] - ref)) <= 1e-4 * rms(ref) + 1e-6
-    ids_o, w_o = oracle.topk_softmax(lg, wl.k)
-    assert np.array_equal(ids.cpu().numpy(), ids_o)
-    assert np.max(np.abs(w.cpu().numpy() - w_o)) <= 1e-6
-    ids_agree(ids.cpu().numpy()[rows], ref, wl.k)
-    # the bias makes the load skewed: the busiest expert far above the mean
+    lg_ref, ids_ref, w_ref = oracle_routes(L, rows)
+    lg = logits.cpu().numpy().astype(np.float64)[rows]
+    err = np.max(np.abs(lg - lg_ref))
+    assert err <= 1e-4 * rms(lg_ref) + 1e-6
+    routes_agree(ids.cpu().numpy()[rows], lg_ref, wl.k, err)
+    # the Zipf bias makes the load skewed: the busiest expert far above the mean
     counts = np.bincount(ids.cpu().numpy().ravel(), minlength=wl.E)
     assert counts.max() > 8 * counts.mean()
 
@@ -120,15 +153,16 @@ def _check_permute(L, ids_np, T):
 
 
 @pytest.mark.parametrize("name", ["tiny", "default", "large", "verify4", "decode1"])
-def test_permute_from_route(name, dev):
+def test_permute_oracle_routes(name, dev):
     L = layer_for(name, dev)
-    ids, _, _ = L.route()
-    _check_permute(L, ids.cpu().numpy(), WORKLOADS[name].T)
+    _, ids, _ = oracle_routes(L, sample(WORKLOADS[name].T, 2048, 9))
+    _check_permute(L, ids, ids.shape[0])
 
 
 @pytest.mark.parametrize("T,E,k,pattern", [
     (1, 16, 4, "random"), (3000, 64, 4, "random"), (300, 16, 4, "same"),
-    (2500, 1024, 32, "random"), (777, 8, 8, "random"), (4097, 5, 1, "skew")])
+    (2500, 1024, 32, "random"), (777, 8, 8, "random"), (4097, 5, 1, "skew"),
+    (6144, 512, 10, "random")])
 def test_permute_patterns(T, E, k, pattern, dev):
     L = Layer.custom(dev, T=1, d=128, E=E, k=k, n=128, group=64, seed=31)
     rng = np.random.default_rng(T + E)
@@ -137,15 +171,14 @@ def test_permute_patterns(T, E, k, pattern, dev):
     elif pattern == "skew":
         ids = np.minimum(rng.geometric(0.7, size=(T, k)) - 1, E - 1)
     else:
-        ids = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+        ids = np.argsort(rng.random((T, E)), axis=1)[:, :k]
     _check_permute(L, ids.astype(np.int32), T)
 
 
 def test_permute_flags_out_of_range_ids(dev):
     L = Layer.custom(dev, T=1, d=128, E=8, k=2, n=128, group=64, seed=32)
     ids = np.array([[0, 1], [8, 2], [3, -1]], np.int32)     # 8 and -1 are out of range
-    t = torch.from_numpy(ids).to(dev)
-    counts, offsets, st, sr = L.permute(t, 3)
+    counts, offsets, st, sr = L.permute(torch.from_numpy(ids).to(dev), 3)
     torch.cuda.synchronize()
     assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
     assert sm.strata_moe_device_status() == sm.STRATA_OK        # cleared
@@ -161,39 +194,64 @@ GEMM_CASES = [("tiny", 10**9), ("default", 10**9), ("large", 384), ("verify4", 1
 def test_expert_gemms(name, max_rows, dev):
     L = layer_for(name, dev)
     wl = WORKLOADS[name]
-    T, S = wl.T, wl.S
-    ids, w, _ = L.route()
-    counts, offsets, st, sr = L.permute(ids, T)
-    h = L.gate_up(L.x, st, offsets, T)
-    scale = torch.linspace(0.5, 1.5, S, device=dev, dtype=torch.float32)
-    rows_scaled = L.down(h, offsets, T, row_scale=scale)
-    rows = L.down(h, offsets, T)
-    assert_device_ok()
-    st_np = st.cpu().numpy()
-    off_np = offsets.cpu().numpy()
-    expert_of_row = np.searchsorted(off_np, np.arange(S), side="right") - 1
+    T, S, k = wl.T, wl.S, wl.k
+    # routes and grouping from the oracle; both sides get the same
+    _, ids, w = oracle_routes(L)
+    counts, offsets, st, sr = oracle.permute(ids, wl.E)
+    off_d = torch.from_numpy(offsets).to(dev)
+    st_d = torch.from_numpy(st).to(dev)
+    expert_of_row = np.searchsorted(offsets, np.arange(S), side="right") - 1
     pick = sample(S, max_rows, 11)
+    rng = np.random.default_rng(12)
+
     # gate/up + SwiGLU on the gathered x rows
-    h_ref = oracle.gate_up_rows(L.inp["x"][st_np[pick]], expert_of_row[pick], L.inp, wl.group)
-    h_np = bf16_host(h)
-    assert gate_error(bf16_to_f64(h_np[pick]), h_ref) <= GATE
-    # down on the GPU's own h rows (bf16), with and without the row scale
-    o_ref = oracle.down_rows(h_np[pick], expert_of_row[pick], L.inp, wl.group)
-    assert gate_error(bf16_to_f64(bf16_host(rows)[pick]), o_ref) <= GATE
-    sc = scale.cpu().numpy()[pick]
-    o_ref_s = oracle.down_rows(h_np[pick], expert_of_row[pick], L.inp, wl.group, sc)
-    assert gate_error(bf16_to_f64(bf16_host(rows_scaled)[pick]), o_ref_s) <= GATE
-    # combine of the GPU rows
-    y = L.combine(rows, w, sr, T)
-    toks = sample(T, 512, 12)
-    y_ref = oracle.combine(bf16_host(rows), w.cpu().numpy().astype(np.float64), sr.cpu().numpy(),
-                           T, wl.k)[toks]
-    y_np = bf16_to_f64(bf16_host(y))[toks]
-    assert np.all(np.abs(y_np - y_ref) <= 2.0 ** -8 * np.abs(y_ref) + 1e-6 * rms(y_ref))
+    h = L.gate_up(L.x, st_d, off_d, T)
+    assert_device_ok()
+    h_ref = oracle.gate_up_rows(L.inp["x"][st[pick]], expert_of_row[pick], L.inp, wl.group)
+    e_h = gate_error(f16_to_f64(f16_host(h)[pick]), h_ref, "fp16")
+    assert e_h <= GATE, e_h
+
+    # down on seeded fp16 rows shaped like h, with and without the row scale
+    h_in = (rng.standard_normal((S, wl.n)) * rms(h_ref)).astype(np.float16)
+    h_in_d = torch.from_numpy(h_in).to(dev)
+    scale = rng.uniform(0.5, 1.5, S).astype(np.float32)
+    rows = L.down(h_in_d, off_d, T)
+    rows_s = L.down(h_in_d, off_d, T, row_scale=torch.from_numpy(scale).to(dev))
+    assert_device_ok()
+    hb = h_in.view(np.uint16)[pick]
+    o_ref = oracle.down_rows(hb, expert_of_row[pick], L.inp, wl.group, a_fp16=True)
+    e_o = gate_error(f16_to_f64(f16_host(rows)[pick]), o_ref, "fp16")
+    assert e_o <= GATE, e_o
+    o_ref_s = oracle.down_rows(hb, expert_of_row[pick], L.inp, wl.group, scale[pick], a_fp16=True)
+    assert gate_error(f16_to_f64(f16_host(rows_s)[pick]), o_ref_s, "fp16") <= GATE
+
+    # combine of seeded fp16 rows with the oracle's weights and slot rows
+    rows_in = (rng.standard_normal((S, wl.d)) * 2).astype(np.float16)
+    y = L.combine(torch.from_numpy(rows_in).to(dev),
+                  torch.from_numpy(w.astype(np.float32)).to(dev),
+                  torch.from_numpy(sr).to(dev), T)
+    assert_device_ok()
+    toks = sample(T, 512, 13)
+    y_ref = oracle.combine(rows_in.view(np.uint16), w.astype(np.float32).astype(np.float64),
+                           sr, T, k, rows_fp16=True)[toks]
+    e_y = gate_error(bf16_to_f64(bf16_host(y))[toks], y_ref, "bf16")
+    # combine alone is exact up to fp32 summation and the final rounding
+    assert e_y <= 1e-5, e_y
+    print(f"{name}: h {e_h:.4f}  rows {e_o:.4f}  combine {e_y:.2e}")
 
 
 # --------------------------------------------------------------------------- whole layer
 FWD_CASES = [("tiny", 64), ("default", 160), ("large", 96), ("verify4", 4), ("decode1", 1)]
+
+
+def _check_forward(L, y, ids, toks, k, group):
+    ref = oracle.moe_forward(L.inp, k, group, tokens=toks)
+    got = bf16_to_f64(bf16_host(y))[toks]
+    err = gate_error(got, ref["y"], "bf16")
+    assert err <= GATE, (err, raw_error(got, ref["y"]))
+    lg_ref = oracle.router_logits(L.inp["x"][toks], L.inp["w_router"], L.inp.get("bias"))
+    ntie, nmis = routes_agree(ids.cpu().numpy()[toks], lg_ref, k, 1e-4 * rms(lg_ref))
+    return err, raw_error(got, ref["y"]), ntie, nmis
 
 
 @pytest.mark.parametrize("name,ntok", FWD_CASES)
@@ -202,13 +260,8 @@ def test_forward(name, ntok, dev):
     wl = WORKLOADS[name]
     y, ids, w = L.forward()
     assert_device_ok()
-    toks = sample(wl.T, ntok, 13)
-    ref = oracle.moe_forward(L.inp, wl.k, wl.group, tokens=toks)
-    err = gate_error(bf16_to_f64(bf16_host(y))[toks], ref["y"])
-    assert err <= GATE, err
-    lg = oracle.router_logits(L.inp["x"][toks], L.inp["w_router"], L.inp.get("bias"))
-    ntie, nmis = ids_agree(ids.cpu().numpy()[toks], lg, wl.k)
-    assert nmis == 0
+    err, raw, ntie, nmis = _check_forward(L, y, ids, sample(wl.T, ntok, 13), wl.k, wl.group)
+    print(f"{name}: gate {err:.4f} raw {raw:.4f} near-ties {ntie} differing routes {nmis}")
 
 
 def test_forward_skewed_chunks(dev):
@@ -219,12 +272,7 @@ def test_forward_skewed_chunks(dev):
     assert_device_ok()
     assert y.shape[0] == wl.T
     assert chunk_sizes(wl.T, wl.chunk) == [6144] * 5 + [3280]
-    toks = sample(wl.T, 96, 14)
-    ref = oracle.moe_forward(L.inp, wl.k, wl.group, tokens=toks)
-    err = gate_error(bf16_to_f64(bf16_host(y))[toks], ref["y"])
-    assert err <= GATE, err
-    lg = oracle.router_logits(L.inp["x"][toks], L.inp["w_router"], L.inp["bias"])
-    ids_agree(ids.cpu().numpy()[toks], lg, wl.k)
+    _check_forward(L, y, ids, sample(wl.T, 96, 14), wl.k, wl.group)
 
 
 EDGE = [
@@ -244,15 +292,12 @@ def test_forward_edge_cases(dims, dev):
     L = Layer.custom(dev, seed=40 + dims["T"], **dims)
     y, ids, w = L.forward()
     assert_device_ok()
-    ref = oracle.moe_forward(L.inp, dims["k"], dims["group"])
-    assert gate_error(bf16_to_f64(bf16_host(y)), ref["y"]) <= GATE
-    lg = oracle.router_logits(L.inp["x"], L.inp["w_router"])
-    ids_agree(ids.cpu().numpy(), lg, dims["k"])
+    _check_forward(L, y, ids, np.arange(dims["T"]), dims["k"], dims["group"])
 
 
 def test_forward_all_tokens_one_expert(dev):
-    """A bias that sends every token to the same experts: 300 rows per expert
-    (three row tiles of the tensor-core kernel) and empty experts elsewhere."""
+    """A bias that sends every token to the same two experts: 300 rows per
+    expert (three row tiles of the tensor-core kernel), the rest empty."""
     L = Layer.custom(dev, T=300, d=256, E=16, k=2, n=256, group=64, seed=50)
     bias = np.zeros(16, np.float32)
     bias[[3, 11]] = 1000.0
@@ -261,17 +306,27 @@ def test_forward_all_tokens_one_expert(dev):
     y, ids, w = L.forward()
     assert_device_ok()
     assert set(np.unique(ids.cpu().numpy())) == {3, 11}
-    ref = oracle.moe_forward(L.inp, 2, 64)
-    assert gate_error(bf16_to_f64(bf16_host(y)), ref["y"]) <= GATE
+    _check_forward(L, y, ids, np.arange(300), 2, 64)
 
 
 def test_zero_scales_give_zero(dev):
-    L = Layer.custom(dev, T=40, d=256, E=8, k=2, n=128, group=64, seed=51)
-    for n in ("gate_s", "up_s", "down_s"):
-        L.w[n].zero_()
-    y, _, _ = L.forward()
-    assert_device_ok()
-    assert torch.count_nonzero(y.float()) == 0
+    for T in (40, 4):
+        L = Layer.custom(dev, T=T, d=256, E=8, k=2, n=128, group=64, seed=51)
+        for n in ("gate_s", "up_s", "down_s"):
+            L.w[n].zero_()
+        y, _, _ = L.forward()
+        assert_device_ok()
+        assert torch.count_nonzero(y.float()) == 0
+
+
+def test_out_of_fp16_range_input_is_reported(dev):
+    L = Layer.custom(dev, T=16, d=128, E=8, k=2, n=128, group=64, seed=53)
+    x = L.x.clone()
+    x[3, 5] = 1.0e6
+    L.forward(x)
+    torch.cuda.synchronize()
+    assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
+    assert sm.strata_moe_device_status() == sm.STRATA_OK
 
 
 def test_token_order_equivariance(dev):
@@ -280,8 +335,8 @@ def test_token_order_equivariance(dev):
     perm = torch.from_numpy(np.random.default_rng(3).permutation(512)).to(dev)
     y_p, ids_p, _ = L.forward(L.x[perm])
     assert torch.equal(ids_p, ids[perm])
-    d = (y_p.float() - y[perm].float()).abs().max().item()
-    assert d <= GATE * y.float().pow(2).mean().sqrt().item()
+    # a token's result depends only on its own row: bit-identical
+    assert torch.equal(y_p, y[perm])
 
 
 def test_chunking_matches_whole_batch(dev):
@@ -334,8 +389,21 @@ def test_empty_batch(dev):
                                  L.q4("down"), dims, y, None, None, None, 0) == sm.STRATA_OK
     counts = torch.full((8,), 7, dtype=torch.int32, device=dev)
     offsets = torch.full((9,), 7, dtype=torch.int32, device=dev)
-    dummy = torch.empty(4, dtype=torch.int32, device=dev)
-    assert sm.strata_moe_permute(dummy, dims, counts, offsets, dummy, dummy, None, 0) == sm.STRATA_OK
+    assert sm.strata_moe_permute(None, dims, counts, offsets, None, None, None, 0) == sm.STRATA_OK
     torch.cuda.synchronize()
     assert int(counts.abs().sum()) == 0 and int(offsets.abs().sum()) == 0
     assert_device_ok()
+
+
+def test_bad_offsets_are_reported_not_used(dev):
+    L = Layer.custom(dev, T=16, d=128, E=8, k=2, n=128, group=64, seed=54)
+    dims = L.dims
+    offsets = torch.tensor([0, 5, 3, 40, 40, 40, 40, 40, 32], dtype=torch.int32, device=dev)
+    st = torch.zeros(32, dtype=torch.int32, device=dev)
+    h = torch.full((32, 128), 7.0, dtype=torch.float16, device=dev)
+    ws = sm.workspace(dims, dev)
+    assert sm.strata_moe_expert_gemm_q4(sm.STRATA_OP_GATE_UP_SWIGLU, L.x, st, offsets,
+                                        L.q4("gate"), L.q4("up"), None, dims, h, ws) == sm.STRATA_OK
+    torch.cuda.synchronize()
+    assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
+    assert bool((h == 7.0).all())                    # nothing was written
