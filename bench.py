@@ -222,6 +222,15 @@ def run_ours(args, wl):
     clk = clocks.stop() if clocks else None
     assert sm.strata_moe_device_status(stream) == sm.STRATA_OK
 
+    if args.only_forward:
+        if world > 1:
+            dist.destroy_process_group()
+        if rank != 0:
+            return None
+        return {"config": {"workload": wl.name}, "ms_per_step": round(total_ms / args.steps, 4),
+                "value": round(T * args.steps * world / (total_ms / 1e3), 1), "unit": "tokens/s",
+                "note": "forward only (profiling run)"}
+
     # ---- breakdown: the same layer as separate entry points, events around each
     ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     wts = torch.empty((T, k), dtype=torch.float32, device=dev)
@@ -397,10 +406,20 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--ref-tokens", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (profiling cases; not a bench line)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E (profiling cases; not a bench line)")
+    ap.add_argument("--only-forward", action="store_true",
+                    help="time the forward only (fewer launches under a profiler)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
+    if args.tokens or args.experts:
+        from moe_inputs import Workload
+        wl = Workload(**{**wl.__dict__, "T": args.tokens or wl.T, "E": args.experts or wl.E,
+                         "name": f"{wl.name}_T{args.tokens or wl.T}_E{args.experts or wl.E}"})
     if wl.chunk and wl.T > wl.chunk:
         # a chunked workload is timed one chunk (the largest) at a time
         from moe_inputs import Workload
