@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(st::THREADS)
       float acc0[4] = {0.f, 0.f, 0.f, 0.f};
       float acc1[4] = {0.f, 0.f, 0.f, 0.f};
 
+      __syncwarp();   // mma.sync.aligned needs the warp converged
       for (int kb0 = 0; kb0 < KB; kb0 += st::UNROLL) {
         uint32_t wa[st::UNROLL][2][2], wb[st::UNROLL][2][2];   // [blk][half][row g / g+8]
         uint4 xa[st::UNROLL][2];

@@ -2,81 +2,126 @@
 // the int4 dequantisation fused into the mainloop.
 //
 // The expert matmul is the heaviest compute of the layer and dequantisation
-// must happen inside it, never as a separate pass that materialises bf16
+// must happen inside it, never as a separate pass that materialises dense
 // weights (kongchang.com "两天移植，预填充提速8倍：Strata引擎实测", section
 // "Strata快在哪" and its MMQ note; lqnn.cn static review, sections 1.2 and
 // 6.2).  The activation is fused with the projection (yfxerp.com review,
-// section 5.1): the gate/up kernel's epilogue applies SwiGLU.
+// section 5.1): the gate/up epilogue applies SwiGLU.
 //
-// Swap-AB formulation, one work unit = (expert e, 128 output features,
-// up to 128 rows of that expert):
-//   A (M = 128)  dequantised weight rows of the expert, K-major, bf16
-//   B (N <= 128) the unit's token rows, K-major, bf16 (gathered x rows for
-//                gate/up, contiguous h rows for down), N rounded up to 16
-//   D (TMEM)     fp32 accumulators, lane = feature, column = row
-// Warp roles (192 threads, persistent CTAs, one per SM):
-//   warp 0     TMA of packed int4 weights (32 B per row per 64-K stage) and
-//              cp.async gather of the B rows straight into the swizzled tile
-//   warp 1     one thread issues tcgen05.mma (kind::f16, fp32 accumulate)
-//   warps 2-5  dequantise packed -> bf16 into the 128-byte-swizzled A tile
-//              (thread = weight row), then run the epilogue of the unit from
-//              TMEM (SwiGLU for gate/up, row scale for down)
-// Operands are fp16 (kind::f16 with f16 A and B): the gathered token rows are
-// an fp16 copy of x (exact for |x| < 65504; made once per call), h is kept in
-// fp16, and each dequantised weight is RNE_fp16(q * s) -- fp16 holds q * s to
-// 2^-11, where bf16 weights (2^-8) would cost the layer most of its error
-// budget.  Dequantisation: q in [-8, 7] becomes the fp16 value 1032 + q by
-// placing the nibble (sign bit flipped) in the mantissa of 1024.0, one fma
-// subtracts 1032 exactly, and one fp16 multiply by the fp16 group scale
-// rounds once.
+// Swap-AB formulation.  One work unit = (expert e, two 128-row weight slots,
+// up to 128 token rows of e):
+//   gate/up: slot 0 = 128 gate rows, slot 1 = the same 128 up rows
+//   down:    slot 0, slot 1 = two consecutive 128-row blocks of W_down
+//   A (M = 128) dequantised weights, fp16, written by threads straight into
+//               tensor memory (tcgen05.st), read by tcgen05.mma from TMEM
+//   B (N <= 128) the unit's token rows, fp16, K-major, 128-byte swizzled in
+//               shared memory (one tile feeds both slots' MMAs)
+//   D           fp32 accumulators in TMEM, lane = weight row, column = token
+// Keeping A out of shared memory leaves shared-memory bandwidth to the B
+// tiles and the packed weights; the MMAs' own reads of B need half of it.
+//
+// Warp roles (480 threads, persistent, one CTA per SM):
+//   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
+//                swizzle) into an 8-deep ring
+//   warp 1       tcgen05.mma issue (one thread)
+//   warp 2       cp.async gather of the unit's token rows into a 6-deep ring
+//   warps 3-10   two dequantising warpgroups taking alternate stages; thread
+//                = weight row; fp16 pairs go to TMEM with tcgen05.st; each
+//                thread loads its row's group scales one own-stage ahead into
+//                registers (plain loads: filling a shared-memory scale ring
+//                with 4-byte cp.async corrupted neighbouring data on B200)
+//   warps 11-14  epilogue: TMEM -> registers -> SwiGLU or row scale -> fp16,
+//                transposed through shared memory into whole-row stores
+// TMEM (512 columns): accumulators of slot 0/1 at columns 0/128, four A
+// stages of 64 columns (32 per slot) at 256..511.
+//
+// Operands are fp16 (kind::f16): x is copied to fp16 once per call (exact for
+// |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
+// keeps q * s to 2^-11, where bf16 weights (2^-8) would use up most of the
+// layer's error budget.  Dequantisation: the nibble with its sign bit flipped
+// goes into the mantissa of 1024.0 (giving 1032 + q), one fma subtracts 1032
+// exactly, one fp16 multiply by the fp16 group scale rounds once.
 #include "common.cuh"
 #include "internal.h"
 
 namespace strata {
 
 namespace tc {
-constexpr int BM = 128;                   // output features per unit (A rows, TMEM lanes)
-constexpr int NT = kTileRows;             // max token rows per unit (B rows, TMEM columns)
-constexpr int BK = 64;                    // K per stage
-constexpr int A_BYTES = BM * BK * 2;      // 16 KB bf16 tile
-constexpr int B_BYTES = NT * BK * 2;      // 16 KB bf16 tile
-constexpr int RAW_BYTES = BM * BK / 2;    //  4 KB packed int4 tile
-constexpr int THREADS = 192;
+constexpr int BM = 128;                    // weight rows per slot (TMEM lanes)
+constexpr int NT = kTileRows;              // token rows per unit (max MMA N)
+constexpr int BK = 64;                     // K per stage
+constexpr int RAW_ST = 8;                  // packed-weight ring depth
+constexpr int B_ST = 6;                    // token-row ring depth
+constexpr int A_ST = 4;                    // TMEM A stages
+constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
+constexpr int B_BYTES = NT * BK * 2;       // 16 KB
+constexpr int EPI_PITCH = 40;              // halves per transpose-tile row (80 B)
 
-template <int NMAT>
-struct Cfg {
-  static constexpr int STAGES = NMAT == 2 ? 3 : 4;
-  static constexpr int TMEM_COLS = NMAT * NT;
-  static constexpr int A_OFF = 0;
-  static constexpr int B_OFF = A_OFF + STAGES * NMAT * A_BYTES;
-  static constexpr int RAW_OFF = B_OFF + STAGES * B_BYTES;
-  static constexpr int BAR_OFF = RAW_OFF + STAGES * NMAT * RAW_BYTES;
-  static constexpr int NBARS = 4 * STAGES + 2;
-  static constexpr int TOK_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int MISC_OFF = TOK_OFF + NT * 4;
-  static constexpr int SMEM = 1024 + MISC_OFF + 64;
-};
+constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3, W_EPI = 11;
+constexpr int THREADS = 15 * 32;
+
+constexpr int RAW_OFF = 0;                                        // [RAW_ST][2][RAW_BYTES]
+constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;           // [B_ST][B_BYTES]
+constexpr int EPI_OFF = B_OFF + B_ST * B_BYTES;                   // [4][32][EPI_PITCH] fp16
+constexpr int EPI_BYTES = 4 * 32 * EPI_PITCH * 2;
+constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
+constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
+constexpr int TOK_OFF = BAR_OFF + NBARS * 8;
+constexpr int MISC_OFF = TOK_OFF + NT * 4;
+constexpr int SMEM = 1024 + MISC_OFF + 64;
+
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t A_COL = 256;
 }  // namespace tc
 
 struct TcArgs {
-  const uint16_t* a;
-  const int32_t* sorted_token;
+  const uint16_t* a;            // B operand rows (fp16): x16 [T][K] or h [S][K]
+  const int32_t* sorted_token;  // gate/up: row -> token
   const int32_t* offsets;
   const int2* tile_table;
-  const int32_t* tile_prefix;
+  const int32_t* total_tiles;   // -> tile_prefix[E]
   const uint16_t* s0;
   const uint16_t* s1;
   const float* row_scale;
   uint16_t* out;
-  int K, N, G;
-  int a_rows;          // rows of `a` (bounds for the gathered token indices)
+  int K, N, G, E;
+  int a_rows;
   unsigned* err;
 };
 
-// 8 int4 (natural order: nibble i = element i) -> 8 fp16 = RNE(q_i * s).
-__device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t sc2) {
+// One work unit, decoded from its index.
+struct Unit {
+  int e, p0, cnt, nrows, nslots;
+  int wrow[2];      // first weight row of each slot in the [E*N] row space
+  int fout[2];      // first output feature of each slot
+};
+
+template <int OP>
+__device__ __forceinline__ Unit decode_unit(const TcArgs& a, int u, int FB) {
+  Unit U;
+  const int2 te = a.tile_table[u / FB];
+  const int fb = u % FB;
+  U.e = te.x;
+  U.p0 = a.offsets[U.e] + te.y * tc::NT;
+  U.cnt = min(tc::NT, a.offsets[U.e + 1] - U.p0);
+  U.nrows = (U.cnt + 15) & ~15;
+  if (OP == 0) {
+    U.nslots = 2;
+    U.fout[0] = U.fout[1] = fb * tc::BM;
+    U.wrow[0] = U.wrow[1] = U.e * a.N + fb * tc::BM;
+  } else {
+    U.fout[0] = fb * 2 * tc::BM;
+    U.fout[1] = U.fout[0] + tc::BM;
+    U.nslots = U.fout[1] < a.N ? 2 : 1;
+    U.wrow[0] = U.e * a.N + U.fout[0];
+    U.wrow[1] = U.wrow[0] + tc::BM;
+  }
+  return U;
+}
+
+// 8 int4 (natural order: nibble i = element i) -> 4 fp16 pairs = RNE(q * s).
+__device__ __forceinline__ void dequant8(uint32_t w, uint32_t sc2, uint32_t* r) {
   const uint32_t w4 = w >> 4;
-  uint32_t r[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     // byte i of w (element 2i in its low nibble) to the low half, byte i of
@@ -89,11 +134,6 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t sc2) {
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o) : "r"(qv), "r"(sc2));
     r[i] = o;
   }
-  return make_uint4(r[0], r[1], r[2], r[3]);
-}
-
-__device__ __forceinline__ uint32_t scale_f16x2(uint16_t s_f16) {
-  return (uint32_t)s_f16 | ((uint32_t)s_f16 << 16);
 }
 
 // fp16 copy of bf16 rows (the gathered B operand of the gate/up GEMM).
@@ -118,75 +158,101 @@ __global__ void __launch_bounds__(256)
   if (over) atomicOr(err, kErrRange);
 }
 
-template <int NMAT>
+template <int OP>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
                           const __grid_constant__ CUtensorMap map_q1, const TcArgs args) {
   using namespace tc;
-  using C = Cfg<NMAT>;
-  constexpr int ST = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = smem + C::A_OFF;     // [ST][NMAT][A_BYTES]
-  uint8_t* sB = smem + C::B_OFF;     // [ST][B_BYTES]
-  uint8_t* sRaw = smem + C::RAW_OFF; // [ST][NMAT][RAW_BYTES]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint8_t* sRaw = smem + RAW_OFF;
+  uint8_t* sB = smem + B_OFF;
+  uint16_t* sEpi = reinterpret_cast<uint16_t*>(smem + EPI_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* raw_full = bars;
-  uint64_t* b_full = bars + ST;
-  uint64_t* a_full = bars + 2 * ST;
-  uint64_t* empty = bars + 3 * ST;
-  uint64_t* acc_full = bars + 4 * ST;
+  uint64_t* raw_empty = raw_full + RAW_ST;
+  uint64_t* b_full = raw_empty + RAW_ST;
+  uint64_t* b_empty = b_full + B_ST;
+  uint64_t* a_full = b_empty + B_ST;
+  uint64_t* a_empty = a_full + A_ST;
+  uint64_t* acc_full = a_empty + A_ST;
   uint64_t* acc_empty = acc_full + 1;
-  int32_t* tok = reinterpret_cast<int32_t*>(smem + C::TOK_OFF);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  int32_t* tok = reinterpret_cast<int32_t*>(smem + TOK_OFF);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int K = args.K, N = args.N;
+  const int K = args.K, N = args.N, G = args.G;
   const int KB = K / BK;
-  const int FB = N / BM;
+  const int FB = OP == 0 ? N / BM : (N + 2 * BM - 1) / (2 * BM);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < RAW_ST; ++s) {
       mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], BM);
+    }
+    for (int s = 0; s < B_ST; ++s) {
       mbar_init(&b_full[s], 32);
-      mbar_init(&a_full[s], 128);
-      mbar_init(&empty[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < A_ST; ++s) {
+      mbar_init(&a_full[s], BM);
+      mbar_init(&a_empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, BM);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == W_TMA && lane == 0) {
     prefetch_tmap(&map_q0);
-    if (NMAT == 2) prefetch_tmap(&map_q1);
+    if (OP == 0) prefetch_tmap(&map_q1);
   }
-  if (warp == 1) tmem_alloc(tmem_holder, C::TMEM_COLS);
+  if (warp == W_MMA) tmem_alloc(tmem_holder, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // total work = tiles x feature blocks (args.tile_prefix points at the
-  // total tile count, entry E of the per-expert prefix)
-  const int units = (*args.tile_prefix) * FB;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  const int units = (*args.total_tiles) * FB;
+  const int my_units =
+      (int)blockIdx.x < units ? (units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int total_stages = my_units * KB;
+
+  if (warp == W_TMA) {
+    // -------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const CUtensorMap* map_slot1 = OP == 0 ? &map_q1 : &map_q0;
+      uint32_t g = 0;
+      bool stop = false;
+      for (int i = 0; i < my_units && !stop; ++i) {
+        const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % RAW_ST;
+          if (g >= (uint32_t)RAW_ST &&
+              !mbar_wait(&raw_empty[s], ((g / RAW_ST) - 1) & 1, abort_flag, args.err)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&raw_full[s], 2 * RAW_BYTES);
+          tma_load_2d(sRaw + (s * 2 + 0) * RAW_BYTES, &map_q0, kb * (BK / 2), U.wrow[0],
+                      &raw_full[s]);
+          tma_load_2d(sRaw + (s * 2 + 1) * RAW_BYTES, map_slot1, kb * (BK / 2), U.wrow[1],
+                      &raw_full[s]);
+        }
+      }
+    }
+  } else if (warp == W_GATHER) {
+    // -------------------------------------------------------------- token-row gather
     uint32_t g = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-      const int2 te = args.tile_table[u / FB];
-      const int fb = u % FB;
-      const int e = te.x;
-      const int p0 = args.offsets[e] + te.y * NT;
-      const int cnt = min(NT, args.offsets[e + 1] - p0);
-      const int nrows = (cnt + 15) & ~15;
+    for (int i = 0; i < my_units && !stop; ++i) {
+      const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
       __syncwarp();
       for (int r = lane; r < NT; r += 32) {
-        int tr = (r < cnt) ? (NMAT == 2 ? args.sorted_token[p0 + r] : p0 + r) : 0;
+        int tr = (r < U.cnt) ? (OP == 0 ? args.sorted_token[U.p0 + r] : U.p0 + r) : 0;
         if ((unsigned)tr >= (unsigned)args.a_rows) {
           atomicOr(args.err, kErrIndex);
           tr = 0;
@@ -194,197 +260,212 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         tok[r] = tr;
       }
       __syncwarp();
-      const int wrow = e * N + fb * BM;
       for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % ST;
-        const uint32_t ph = (g / ST) & 1u;
-        if (g >= (uint32_t)ST && !mbar_wait(&empty[s], ph ^ 1u, abort_flag, args.err)) {
+        const int s = g % B_ST;
+        if (g >= (uint32_t)B_ST &&
+            !mbar_wait(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
           stop = true;
           break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[s], NMAT * RAW_BYTES);
-          tma_load_2d(sRaw + (s * NMAT + 0) * RAW_BYTES, &map_q0, kb * (BK / 2), wrow,
-                      &raw_full[s]);
-          if (NMAT == 2)
-            tma_load_2d(sRaw + (s * NMAT + 1) * RAW_BYTES, &map_q1, kb * (BK / 2), wrow,
-                        &raw_full[s]);
-        }
         const uint32_t bbase = smem_addr(sB + s * B_BYTES);
         const uint16_t* abase = args.a + (size_t)kb * BK;
-        for (int idx = lane; idx < nrows * 8; idx += 32) {
+        for (int idx = lane; idx < U.nrows * 8; idx += 32) {
           const int r = idx >> 3, c = idx & 7;
-          const uint16_t* src = abase + (size_t)tok[r] * K + c * 8;
-          cp_async_16(bbase + sw128_offset(r, c), src, r < cnt ? 16u : 0u);
+          cp_async_16(bbase + sw128_offset(r, c), abase + (size_t)tok[r] * K + c * 8,
+                      r < U.cnt ? 16u : 0u);
         }
         cp_async_arrive(&b_full[s]);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
+  } else if (warp == W_MMA) {
+    // -------------------------------------------------------------- MMA issue
     if (lane == 0) {
       uint32_t g = 0;
-      int i = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < units && !stop; u += gridDim.x, ++i) {
-        const int2 te = args.tile_table[u / FB];
-        const int e = te.x;
-        const int p0 = args.offsets[e] + te.y * NT;
-        const int cnt = min(NT, args.offsets[e + 1] - p0);
-        const int nrows = (cnt + 15) & ~15;
-        const uint32_t idesc = idesc_f32acc(BM, nrows, kFmtF16, 0);
+      for (int i = 0; i < my_units && !stop; ++i) {
+        const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+        const uint32_t idesc = idesc_f32acc(BM, U.nrows, kFmtF16, 0);
         if (i > 0) {
           if (!mbar_wait(acc_empty, (i - 1) & 1, abort_flag, args.err)) break;
           tc_fence_after();
         }
         for (int kb = 0; kb < KB; ++kb, ++g) {
-          const int s = g % ST;
-          const uint32_t ph = (g / ST) & 1u;
-          if (!mbar_wait(&a_full[s], ph, abort_flag, args.err) ||
-              !mbar_wait(&b_full[s], ph, abort_flag, args.err)) {
+          const int sa = g % A_ST, sb = g % B_ST;
+          if (!mbar_wait(&a_full[sa], (g / A_ST) & 1, abort_flag, args.err) ||
+              !mbar_wait(&b_full[sb], (g / B_ST) & 1, abort_flag, args.err)) {
             stop = true;
             break;
           }
-          fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t b0 = smem_addr(sB + s * B_BYTES);
+          fence_proxy_async_smem();
+          const uint32_t b0 = smem_addr(sB + sb * B_BYTES);
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t bd = desc_kmajor_sw128(b0 + ks * 32);
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-              const uint64_t ad =
-                  desc_kmajor_sw128(smem_addr(sA + (s * NMAT + m) * A_BYTES) + ks * 32);
-              mma_f16kind_ss(tmem + m * NT, ad, bd, idesc, (kb | ks) != 0);
+            for (int m = 0; m < 2; ++m) {
+              if (m < U.nslots)
+                mma_f16kind_ts(tmem + m * BM, tmem + A_COL + sa * 64 + m * 32 + ks * 8, bd,
+                               idesc, (kb | ks) != 0);
             }
           }
-          mma_commit(&empty[s]);
+          mma_commit(&a_empty[sa]);
+          mma_commit(&b_empty[sb]);
         }
         if (!stop) mma_commit(acc_full);
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ dequant + epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = q * 32 + lane;            // weight row of this thread
-    const int G = args.G;
-    uint32_t g = 0;
-    int i = 0;
-    bool stop = false;
-    for (int u = blockIdx.x; u < units && !stop; u += gridDim.x, ++i) {
-      const int2 te = args.tile_table[u / FB];
-      const int fb = u % FB;
-      const int e = te.x;
-      const int p0 = args.offsets[e] + te.y * NT;
-      const int cnt = min(NT, args.offsets[e + 1] - p0);
-      const size_t wrow = (size_t)e * N + fb * BM + r;
-      const uint16_t* srow0 = args.s0 + wrow * (K / G);
-      const uint16_t* srow1 = NMAT == 2 ? args.s1 + wrow * (K / G) : nullptr;
-      for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % ST;
-        const uint32_t ph = (g / ST) & 1u;
-        // scales of the (at most two) groups this 64-wide stage touches
-        const int g0 = (kb * BK) / G;
-        const int g1 = (kb * BK + BK / 2) / G;
-        uint32_t sc[NMAT][2];
-        sc[0][0] = scale_f16x2(__ldg(srow0 + g0));
-        sc[0][1] = scale_f16x2(__ldg(srow0 + g1));
-        if (NMAT == 2) {
-          sc[NMAT - 1][0] = scale_f16x2(__ldg(srow1 + g0));
-          sc[NMAT - 1][1] = scale_f16x2(__ldg(srow1 + g1));
-        }
-        if (!mbar_wait(&raw_full[s], ph, abort_flag, args.err)) {
-          stop = true;
-          break;
-        }
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          const uint4* rp = reinterpret_cast<const uint4*>(sRaw + (s * NMAT + m) * RAW_BYTES + r * 32);
-          const uint4 lo = rp[0], hi = rp[1];
-          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          uint8_t* tile = sA + (s * NMAT + m) * A_BYTES;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 o = dequant8(words[c], sc[m][c >> 2]);
-            *reinterpret_cast<uint4*>(tile + sw128_offset(r, c)) = o;
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&a_full[s]);
+  } else if (warp < W_EPI) {
+    // -------------------------------------------------------------- dequantise
+    const int wg = (warp - W_DQ) >> 2;       // takes the stages g with g % 2 == wg
+    const int q = warp & 3;                  // TMEM lane quadrant
+    const int r = q * 32 + lane;             // weight row within the slot
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    const int g_shift = G == 32 ? 5 : (G == 64 ? 6 : 7);
+    int pf_i = -1;
+    Unit pf_U;
+    // Scales of stage gs for this row (both slots; with 32-wide groups the
+    // stage spans two groups): sc[m][0], sc[m][1] as fp16 bits.
+    auto load_scales = [&](int gs, uint32_t (&sc)[2][2]) {
+      if (gs >= total_stages) return;
+      const int i = gs / KB, kb = gs - i * KB;
+      if (i != pf_i) {
+        pf_U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+        pf_i = i;
       }
-      if (stop) break;
-      // ---- epilogue of this unit
-      bool ok = mbar_wait(acc_full, i & 1, abort_flag, args.err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const int feat = fb * BM + r;
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
-      const int nch = (cnt + 31) >> 5;
-      for (int c = 0; c < nch; ++c) {
-        uint32_t acc0[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, acc0);
-        if (NMAT == 2) {
-          uint32_t acc1[32];
-          tmem_ld_32x32b_x32(tbase + NT + c * 32, acc1);
-          tmem_ld_wait();
+      const int grp = (kb * BK) >> g_shift;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int p = c * 32 + j;
-            if (p < cnt) {
-              const float gv = __uint_as_float(acc0[j]);
-              const float uv = __uint_as_float(acc1[j]);
-              const float h = gv / (1.0f + __expf(-gv)) * uv;
-              args.out[(size_t)(p0 + p) * N + feat] = f16_bits(h);
-            }
-          }
+      for (int m = 0; m < 2; ++m) {
+        const uint16_t* sp = (OP == 0 && m == 1) ? args.s1 : args.s0;
+        if (m < pf_U.nslots) {
+          const uint16_t* p = sp + (size_t)(pf_U.wrow[m] + r) * (K / G) + grp;
+          sc[m][0] = __ldg(p);
+          sc[m][1] = G == 32 ? __ldg(p + 1) : sc[m][0];
         } else {
-          tmem_ld_wait();
+          sc[m][0] = sc[m][1] = 0;
+        }
+      }
+    };
+    uint32_t sc_next[2][2] = {{0, 0}, {0, 0}};
+    load_scales(wg, sc_next);
+    for (int j = 0;; ++j) {
+      const int g = wg + 2 * j;
+      if (g >= total_stages) break;
+      // the loads of this stage's scales were issued a whole own stage ago
+      const uint32_t sc_cur[2][2] = {{sc_next[0][0], sc_next[0][1]}, {sc_next[1][0], sc_next[1][1]}};
+      load_scales(g + 2, sc_next);
+      const int sr = g % RAW_ST, sa = g % A_ST;
+      if (!mbar_wait(&raw_full[sr], (g / RAW_ST) & 1, abort_flag, args.err)) break;
+      // packed words of this row; 32-byte swizzle puts chunk c at c ^ ((r >> 2) & 1)
+      uint4 raw[2][2];
+      const int sw = (r >> 2) & 1;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int p = c * 32 + j;
-            if (p < cnt) {
-              float v = __uint_as_float(acc0[j]);
-              if (args.row_scale) v *= args.row_scale[p0 + p];
-              args.out[(size_t)(p0 + p) * N + feat] = f16_bits(v);
+      for (int m = 0; m < 2; ++m) {
+        const uint8_t* rowp = sRaw + (sr * 2 + m) * RAW_BYTES + r * 32;
+        raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * sw);
+        raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * (sw ^ 1));
+      }
+      mbar_arrive(&raw_empty[sr]);
+      if (g >= A_ST && !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
+        break;
+      __syncwarp();       // converged before the .sync.aligned TMEM stores
+      tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t sc_a = sc_cur[m][0] | (sc_cur[m][0] << 16);
+        const uint32_t sc_b = sc_cur[m][1] | (sc_cur[m][1] << 16);
+        const uint32_t words[8] = {raw[m][0].x, raw[m][0].y, raw[m][0].z, raw[m][0].w,
+                                   raw[m][1].x, raw[m][1].y, raw[m][1].z, raw[m][1].w};
+        uint32_t out[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
+        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&a_full[sa]);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    uint16_t* tile = sEpi + (warp - W_EPI) * 32 * EPI_PITCH;
+    for (int i = 0; i < my_units; ++i) {
+      const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+      if (!mbar_wait_warp(acc_full, i & 1, abort_flag, args.err)) break;
+      tc_fence_after();
+      const int nch = (U.cnt + 31) >> 5;
+      for (int m = 0; m < (OP == 0 ? 1 : U.nslots); ++m) {
+        for (int c = 0; c < nch; ++c) {
+          __syncwarp();   // converged before the .sync.aligned TMEM loads
+          uint32_t a0[32];
+          tmem_ld_32x32b_x32(t_lane + m * BM + c * 32, a0);
+          if (OP == 0) {
+            uint32_t a1[32];
+            tmem_ld_32x32b_x32(t_lane + BM + c * 32, a1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
+              tile[j * EPI_PITCH + lane] = f16_bits(gv / (1.0f + __expf(-gv)) * uv);
+            }
+          } else {
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float v = __uint_as_float(a0[j]);
+              const int p = U.p0 + c * 32 + j;
+              if (args.row_scale && c * 32 + j < U.cnt) v *= args.row_scale[p];
+              tile[j * EPI_PITCH + lane] = f16_bits(v);
             }
           }
+          __syncwarp();
+          // thread `lane` writes token row c*32 + lane: this warp's 32 features
+          if (c * 32 + lane < U.cnt) {
+            const uint4* src = reinterpret_cast<const uint4*>(tile + lane * EPI_PITCH);
+            uint4* dst = reinterpret_cast<uint4*>(
+                args.out + (size_t)(U.p0 + c * 32 + lane) * N + U.fout[m] + q * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = src[v];
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
     }
+    (void)r;
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == W_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
 static int g_num_sms = 0;
 
-template <int NMAT>
+template <int OP>
 static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
-  using C = tc::Cfg<NMAT>;
   CUtensorMap m0, m1;
   const uint64_t rows = (uint64_t)p.E * p.N;
   if (encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q0, p.K / 2, rows, p.K / 2,
-                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   m1 = m0;
-  if (NMAT == 2 &&
+  if (OP == 0 &&
       encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q1, p.K / 2, rows, p.K / 2,
-                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<NMAT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM);
     if (e != cudaSuccess) return e;
   }
   if (g_num_sms == 0) {
@@ -393,7 +474,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
     cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (g_num_sms <= 0) g_num_sms = 148;
   }
-  if (p.op == 0) {
+  if (OP == 0) {
     // the gate/up B operand is the fp16 copy of x
     const size_t n8 = (size_t)p.T * p.K / 8;
     int blocks = (int)((n8 + 255) / 256);
@@ -402,11 +483,11 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                                               reinterpret_cast<uint4*>(p.a16), n8, p.err);
   }
   TcArgs a;
-  a.a = p.op == 0 ? p.a16 : p.a;
+  a.a = OP == 0 ? p.a16 : p.a;
   a.sorted_token = p.sorted_token;
   a.offsets = p.offsets;
   a.tile_table = sch.tile_table;
-  a.tile_prefix = sch.tile_prefix + p.E;     // -> total tile count
+  a.total_tiles = sch.tile_prefix + p.E;
   a.s0 = p.s0;
   a.s1 = p.s1;
   a.row_scale = p.row_scale;
@@ -414,16 +495,18 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   a.K = p.K;
   a.N = p.N;
   a.G = p.G;
-  a.a_rows = p.op == 0 ? p.T : p.S;
+  a.E = p.E;
+  a.a_rows = OP == 0 ? p.T : p.S;
   a.err = p.err;
-  const int max_units = max_tiles(p.S, p.E) * (p.N / tc::BM);
-  const int grid = max_units < g_num_sms ? max_units : g_num_sms;
-  moe_gemm_q4_tc_kernel<NMAT><<<grid, tc::THREADS, C::SMEM, s>>>(m0, m1, a);
+  const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
+  const long max_units = (long)max_tiles(p.S, p.E) * FB;
+  const int grid = (int)(max_units < g_num_sms ? max_units : g_num_sms);
+  moe_gemm_q4_tc_kernel<OP><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
-  return p.op == 0 ? launch_tc_impl<2>(p, sch, s) : launch_tc_impl<1>(p, sch, s);
+  return p.op == 0 ? launch_tc_impl<0>(p, sch, s) : launch_tc_impl<1>(p, sch, s);
 }
 
 }  // namespace strata

@@ -108,12 +108,12 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     const int q = warp & 3;          // TMEM lane quadrant this warp may read
     const int row = q * 32 + lane;
     const int t = m0 + row;
-    bool ok = mbar_wait(accf, 0, abort_flag, err);
-    ok = __all_sync(0xffffffffu, ok);
+    const bool ok = mbar_wait_warp(accf, 0, abort_flag, err);
     tc_fence_after();
     if (ok) {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
+        __syncwarp();   // converged before the .sync.aligned TMEM load
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + c * 32, r);
         tmem_ld_wait();

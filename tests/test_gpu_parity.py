@@ -204,9 +204,11 @@ def test_expert_gemms(name, max_rows, dev):
     pick = sample(S, max_rows, 11)
     rng = np.random.default_rng(12)
 
-    # gate/up + SwiGLU on the gathered x rows
+    # gate/up + SwiGLU on the gathered x rows; twice, bit-identical
     h = L.gate_up(L.x, st_d, off_d, T)
+    h2 = L.gate_up(L.x, st_d, off_d, T)
     assert_device_ok()
+    assert torch.equal(h, h2), int((h != h2).sum())
     h_ref = oracle.gate_up_rows(L.inp["x"][st[pick]], expert_of_row[pick], L.inp, wl.group)
     e_h = gate_error(f16_to_f64(f16_host(h)[pick]), h_ref, "fp16")
     assert e_h <= GATE, e_h
