@@ -153,6 +153,24 @@ def profiled_traffic(kernel):
     return e.get("dram_bytes_per_launch")
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(v, device=None):
+    """Maximum of a per-rank float over all ranks (identity without a process
+    group).  The timed region's duration is taken this way."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, max_ms):
+    """Whole-job tokens/s: tokens of all ranks over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- our arm
 def run_ours(args, wl):
     import torch
@@ -193,13 +211,6 @@ def run_ours(args, wl):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---- headline: K forwards, device time
     for _ in range(args.warmup):
         forward()
@@ -217,7 +228,7 @@ def run_ours(args, wl):
         step_ev[i + 1].record(stream)
     ev1.record(stream)
     barrier()
-    total_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    total_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     step_ms = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
     clk = clocks.stop() if clocks else None
     assert sm.strata_moe_device_status(stream) == sm.STRATA_OK
@@ -228,7 +239,8 @@ def run_ours(args, wl):
         if rank != 0:
             return None
         return {"config": {"workload": wl.name}, "ms_per_step": round(total_ms / args.steps, 4),
-                "value": round(T * args.steps * world / (total_ms / 1e3), 1), "unit": "tokens/s",
+                "value": round(job_throughput(T * args.steps, world, total_ms), 1),
+                "unit": "tokens/s",
                 "note": "forward only (profiling run)"}
 
     # ---- breakdown: the same layer as separate entry points, events around each
@@ -287,7 +299,7 @@ def run_ours(args, wl):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -296,7 +308,7 @@ def run_ours(args, wl):
 
     hbm, tf_burst, tf_sus, peak_kind = measured_peaks()
     tokens = T * args.steps * world
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(T * args.steps, world, total_ms)
     ms_step = total_ms / args.steps
     tensor_bound = T > 8
     if tensor_bound:

@@ -24,7 +24,13 @@
 //   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
 //                swizzle) into an 8-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
-//   warp 2       cp.async gather of the unit's token rows into a 6-deep ring
+//   warp 2       token rows into a 6-deep ring, one TMA tile of 128 rows per
+//                stage: the down projection reads h, whose rows are already
+//                grouped by expert; for gate/up a pre-pass writes the fp16 rows
+//                of x in grouped order (x[sorted_token[p]]), so both operands
+//                of every stage arrive by TMA.  (Filling the same shared memory
+//                with cp.async while TMA wrote beside it gave run-to-run
+//                differences on B200; TMA-only staging is deterministic.)
 //   warps 3-10   two dequantising warpgroups taking alternate stages; thread
 //                = weight row; fp16 pairs go to TMEM with tcgen05.st; each
 //                thread loads its row's group scales one own-stage ahead into
@@ -35,8 +41,8 @@
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/128, four A
 // stages of 64 columns (32 per slot) at 256..511.
 //
-// Operands are fp16 (kind::f16): x is copied to fp16 once per call (exact for
-// |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
+// Operands are fp16 (kind::f16): x rows are copied to fp16 in grouped order
+// once per call (exact for |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
 // keeps q * s to 2^-11, where bf16 weights (2^-8) would use up most of the
 // layer's error budget.  Dequantisation: the nibble with its sign bit flipped
 // goes into the mantissa of 1024.0 (giving 1032 + q), one fma subtracts 1032
@@ -136,15 +142,24 @@ __device__ __forceinline__ void dequant8(uint32_t w, uint32_t sc2, uint32_t* r) 
   }
 }
 
-// fp16 copy of bf16 rows (the gathered B operand of the gate/up GEMM).
-// Values beyond the fp16 range become +-inf and are reported as kErrRange.
+// Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]) for the S grouped rows.
+// Out-of-range token indices are reported (kErrIndex) and read row 0; values
+// beyond the fp16 range become +-inf and are reported as kErrRange.
 __global__ void __launch_bounds__(256)
-    bf16_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n8,
-                       unsigned* err) {
-  bool over = false;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+    gather_rows_f16_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
+                           int T, int d, int S, uint16_t* __restrict__ xs, unsigned* err) {
+  const int cpr = d / 8;                      // 16-byte chunks per row
+  const size_t n = (size_t)S * cpr;
+  bool over = false, bad = false;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
-    const uint4 v = src[i];
+    const int p = (int)(i / cpr), c = (int)(i - (size_t)p * cpr);
+    int t = sorted_token[p];
+    if ((unsigned)t >= (unsigned)T) {
+      bad = true;
+      t = 0;
+    }
+    const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8);
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[4];
 #pragma unroll
@@ -153,15 +168,17 @@ __global__ void __launch_bounds__(256)
       over |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
       out[j] = (uint32_t)f16_bits(lo) | ((uint32_t)f16_bits(hi) << 16);
     }
-    dst[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(xs + (size_t)p * d + c * 8) = make_uint4(out[0], out[1], out[2], out[3]);
   }
   if (over) atomicOr(err, kErrRange);
+  if (bad) atomicOr(err, kErrIndex);
 }
 
 template <int OP>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
-                          const __grid_constant__ CUtensorMap map_q1, const TcArgs args) {
+                          const __grid_constant__ CUtensorMap map_q1,
+                          const __grid_constant__ CUtensorMap map_b, const TcArgs args) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -178,7 +195,6 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   uint64_t* a_empty = a_full + A_ST;
   uint64_t* acc_full = a_empty + A_ST;
   uint64_t* acc_empty = acc_full + 1;
-  int32_t* tok = reinterpret_cast<int32_t*>(smem + TOK_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
 
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       mbar_init(&raw_empty[s], BM);
     }
     for (int s = 0; s < B_ST; ++s) {
-      mbar_init(&b_full[s], 32);
+      mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
     for (int s = 0; s < A_ST; ++s) {
@@ -209,6 +225,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   if (warp == W_TMA && lane == 0) {
     prefetch_tmap(&map_q0);
     if (OP == 0) prefetch_tmap(&map_q1);
+    prefetch_tmap(&map_b);
   }
   if (warp == W_MMA) tmem_alloc(tmem_holder, TMEM_COLS);
   tc_fence_before();
@@ -245,36 +262,24 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       }
     }
   } else if (warp == W_GATHER) {
-    // -------------------------------------------------------------- token-row gather
-    uint32_t g = 0;
-    bool stop = false;
-    for (int i = 0; i < my_units && !stop; ++i) {
-      const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
-      __syncwarp();
-      for (int r = lane; r < NT; r += 32) {
-        int tr = (r < U.cnt) ? (OP == 0 ? args.sorted_token[U.p0 + r] : U.p0 + r) : 0;
-        if ((unsigned)tr >= (unsigned)args.a_rows) {
-          atomicOr(args.err, kErrIndex);
-          tr = 0;
+    // -------------------------------------------------------------- token rows (B)
+    // one TMA tile of 128 grouped rows per stage (rows past the unit belong
+    // to other units or lie beyond S; the MMA reads only nrows of them)
+    if (lane == 0) {
+      uint32_t g = 0;
+      bool stop = false;
+      for (int i = 0; i < my_units && !stop; ++i) {
+        const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % B_ST;
+          if (g >= (uint32_t)B_ST &&
+              !mbar_wait(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[s], B_BYTES);
+          tma_load_2d(sB + s * B_BYTES, &map_b, kb * BK, U.p0, &b_full[s]);
         }
-        tok[r] = tr;
-      }
-      __syncwarp();
-      for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % B_ST;
-        if (g >= (uint32_t)B_ST &&
-            !mbar_wait(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
-          stop = true;
-          break;
-        }
-        const uint32_t bbase = smem_addr(sB + s * B_BYTES);
-        const uint16_t* abase = args.a + (size_t)kb * BK;
-        for (int idx = lane; idx < U.nrows * 8; idx += 32) {
-          const int r = idx >> 3, c = idx & 7;
-          cp_async_16(bbase + sw128_offset(r, c), abase + (size_t)tok[r] * K + c * 8,
-                      r < U.cnt ? 16u : 0u);
-        }
-        cp_async_arrive(&b_full[s]);
       }
     }
   } else if (warp == W_MMA) {
@@ -297,7 +302,6 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             break;
           }
           tc_fence_after();
-          fence_proxy_async_smem();
           const uint32_t b0 = smem_addr(sB + sb * B_BYTES);
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
@@ -458,6 +462,13 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   m1 = m0;
+  // B rows: grouped fp16 rows [S][K] (the gathered copy of x, or h)
+  CUtensorMap mb;
+  const uint16_t* brows = OP == 0 ? p.a16 : p.a;
+  if (encode_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, brows, p.K, p.S, (uint64_t)p.K * 2,
+                     tc::BK, tc::NT, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   if (OP == 0 &&
       encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q1, p.K / 2, rows, p.K / 2,
                      tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
@@ -475,15 +486,15 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
     if (g_num_sms <= 0) g_num_sms = 148;
   }
   if (OP == 0) {
-    // the gate/up B operand is the fp16 copy of x
-    const size_t n8 = (size_t)p.T * p.K / 8;
-    int blocks = (int)((n8 + 255) / 256);
-    if (blocks > 8 * g_num_sms) blocks = 8 * g_num_sms;
-    bf16_to_f16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(p.a),
-                                              reinterpret_cast<uint4*>(p.a16), n8, p.err);
+    // the gate/up B operand: fp16 rows of x in grouped order
+    const size_t n = (size_t)p.S * (p.K / 8);
+    long blocks = (long)((n + 255) / 256);
+    if (blocks > 16L * g_num_sms) blocks = 16L * g_num_sms;
+    gather_rows_f16_kernel<<<(int)blocks, 256, 0, s>>>(p.a, p.sorted_token, p.T, p.K, p.S, p.a16,
+                                                       p.err);
   }
   TcArgs a;
-  a.a = OP == 0 ? p.a16 : p.a;
+  a.a = brows;
   a.sorted_token = p.sorted_token;
   a.offsets = p.offsets;
   a.tile_table = sch.tile_table;
@@ -501,7 +512,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < g_num_sms ? max_units : g_num_sms);
-  moe_gemm_q4_tc_kernel<OP><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, a);
+  moe_gemm_q4_tc_kernel<OP><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
   return cudaGetLastError();
 }
 
