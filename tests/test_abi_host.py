@@ -58,9 +58,10 @@ LARGE = dict(T=6144, d=4096, E=512, k=10, n=1024, group=64)
 def test_workspace_bytes():
     n = sm.strata_moe_workspace_bytes(LARGE)
     S = 6144 * 10
-    # at least the two per-row intermediates h [S][n] and rows [S][d] in bf16
-    assert n >= S * 1024 * 2 + S * 4096 * 2
-    assert n < S * 1024 * 2 + S * 4096 * 2 + 64 * 2 ** 20
+    # at least the per-row fp16 buffers: grouped x [S][d], h [S][n], rows [S][d]
+    rows = S * 4096 * 2 + S * 1024 * 2 + S * 4096 * 2
+    assert n >= rows
+    assert n < rows + 64 * 2 ** 20
     assert n % 256 == 0
     assert sm.strata_moe_workspace_bytes(dict(LARGE, T=1)) < 4 * 2 ** 20
     assert sm.strata_moe_workspace_bytes(dict(LARGE, T=0)) >= 0
