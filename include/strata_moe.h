@@ -165,6 +165,38 @@ STRATA_API strata_status_t strata_moe_permute(const int32_t* topk_ids,
                                    int32_t* slot_row, void* ws, size_t ws_bytes,
                                    strata_stream_t stream);
 
+/* strata_moe_permute without a caller workspace.  The pages describe no such
+ * call: it exists for callers that cannot hand the library device memory --
+ * a host program that owns only the five tensors it passes (it has no device
+ * allocator of its own to carve a workspace from), or a deployment that
+ * budgets every device byte up front and forbids allocation once serving
+ * starts.  Such callers get the same result as strata_moe_permute (bit for
+ * bit: same kernels, same order) with the per-chunk histogram held in a
+ * fixed scratch array compiled into the library, one per device.  Nothing is
+ * allocated or freed: no cudaMalloc/cudaFree and no allocating library call,
+ * on the first call or later.
+ *   Arguments and outputs: as strata_moe_permute, minus ws/ws_bytes.
+ *   Limit: the scratch holds STRATA_PERMUTE_STATIC_SCRATCH_INTS int32
+ *     values (512 KiB); a call needs ceil(T*k / 1024) * E of them (E = 512:
+ *     T*k up to 262144 slots; E = 1024: up to 131072).  Larger inputs return
+ *     STRATA_ERR_WORKSPACE before anything is launched.
+ *   Zero state: none -- every scratch value a call reads was written earlier
+ *     in the same call, so the scratch needs no clearing, and nothing carries
+ *     over from one call to the next.
+ *   Setup: the first call on each device looks up the scratch's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches it;
+ *     that lookup may synchronise with the device, so make the first call on
+ *     a device before any stream capture begins.
+ *   Concurrency: all calls on one device share the one scratch array.  Two
+ *     calls in flight at the same time on the same device (different
+ *     streams, or different host threads without ordering) race on it and
+ *     produce wrong groupings; order them on one stream or with events. */
+#define STRATA_PERMUTE_STATIC_SCRATCH_INTS 131072
+STRATA_API strata_status_t strata_moe_permute_static(const int32_t* topk_ids,
+                                          strata_moe_dims_t dims, int32_t* counts,
+                                          int32_t* offsets, int32_t* sorted_token,
+                                          int32_t* slot_row, strata_stream_t stream);
+
 /* Grouped expert projection with int4 dequantisation fused into the GEMM
  * (dequantise inside the matmul: lqnn.cn review 1.2 / 6.2; expert matmul is
  * the heaviest compute: kongchang.com page, "Strata快在哪"; activation fused

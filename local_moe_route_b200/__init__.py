@@ -20,7 +20,8 @@ __all__ = [
     "STRATA_ERR_CUDA", "STRATA_ERR_DEVICE_CHECK", "STRATA_OP_GATE_UP_SWIGLU", "STRATA_OP_DOWN",
     "Dims", "Q4", "StrataError", "lib", "lib_path", "check",
     "strata_moe_workspace_bytes", "strata_status_string", "strata_moe_route",
-    "strata_moe_permute", "strata_moe_expert_gemm_q4", "strata_moe_combine",
+    "strata_moe_permute", "strata_moe_permute_static", "STRATA_PERMUTE_STATIC_SCRATCH_INTS",
+    "strata_moe_expert_gemm_q4", "strata_moe_combine",
     "strata_moe_forward", "strata_moe_device_status", "workspace",
 ]
 
@@ -32,6 +33,7 @@ STRATA_ERR_CUDA = 4
 STRATA_ERR_DEVICE_CHECK = 5
 STRATA_OP_GATE_UP_SWIGLU = 0
 STRATA_OP_DOWN = 1
+STRATA_PERMUTE_STATIC_SCRATCH_INTS = 131072
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libstrata_moe.so"
@@ -95,6 +97,8 @@ def lib() -> ctypes.CDLL:
     L.strata_moe_route.restype = st
     L.strata_moe_permute.argtypes = [vp, Dims, vp, vp, vp, vp, vp, sz, vp]
     L.strata_moe_permute.restype = st
+    L.strata_moe_permute_static.argtypes = [vp, Dims, vp, vp, vp, vp, vp]
+    L.strata_moe_permute_static.restype = st
     L.strata_moe_expert_gemm_q4.argtypes = [st, vp, vp, vp, Q4, Q4, vp, Dims, vp, vp, sz, vp]
     L.strata_moe_expert_gemm_q4.restype = st
     L.strata_moe_combine.argtypes = [vp, vp, vp, Dims, vp, vp]
@@ -160,6 +164,13 @@ def strata_moe_permute(topk_ids, dims, counts, offsets, sorted_token, slot_row, 
         _ptr(topk_ids), Dims.of(dims), _ptr(counts), _ptr(offsets), _ptr(sorted_token),
         _ptr(slot_row), _ptr(ws), _nbytes(ws) if ws_bytes is None else int(ws_bytes),
         _stream(stream))
+
+
+def strata_moe_permute_static(topk_ids, dims, counts, offsets, sorted_token, slot_row,
+                              stream=None) -> int:
+    return lib().strata_moe_permute_static(
+        _ptr(topk_ids), Dims.of(dims), _ptr(counts), _ptr(offsets), _ptr(sorted_token),
+        _ptr(slot_row), _stream(stream))
 
 
 def strata_moe_expert_gemm_q4(op, a, sorted_token, offsets, w0, w1, row_scale, dims, out,

@@ -264,6 +264,53 @@ strata_status_t strata_moe_permute(const int32_t* topk_ids, strata_moe_dims_t di
                                     sorted_token, slot_row, static_cast<int32_t*>(ws), err, s));
 }
 
+// Fixed scratch for strata_moe_permute_static: the per-chunk histogram of
+// the grouping, sized once at compile time so that callers without a device
+// allocator can group slots.  One copy per device (a __device__ variable).
+static __device__ __align__(256) int32_t g_permute_scratch[STRATA_PERMUTE_STATIC_SCRATCH_INTS];
+
+// Device address of g_permute_scratch on the current device, looked up once
+// per device and cached (nullptr if the lookup fails).
+static int32_t* permute_scratch_ptr() {
+  static std::mutex mu;
+  static int32_t* cache[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int32_t*>(p);
+  }
+  return cache[dev];
+}
+
+strata_status_t strata_moe_permute_static(const int32_t* topk_ids, strata_moe_dims_t dims,
+                                          int32_t* counts, int32_t* offsets,
+                                          int32_t* sorted_token, int32_t* slot_row,
+                                          strata_stream_t stream) {
+  strata_status_t st = check_dims(dims);
+  if (st != STRATA_OK) return st;
+  if (!ok_ptr(counts) || !ok_ptr(offsets)) return STRATA_ERR_INVALID_ARG;
+  // The scratch limit is checked before any CUDA call, so an oversized input
+  // is rejected without touching the device.
+  if (permute_scratch(dims) > sizeof(int32_t) * (size_t)STRATA_PERMUTE_STATIC_SCRATCH_INTS)
+    return STRATA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dims.T == 0) {
+    if (cudaMemsetAsync(counts, 0, (size_t)dims.E * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, (size_t)(dims.E + 1) * 4, s) != cudaSuccess)
+      return STRATA_ERR_CUDA;
+    return STRATA_OK;
+  }
+  if (!ok_ptr(topk_ids) || !ok_ptr(sorted_token) || !ok_ptr(slot_row)) return STRATA_ERR_INVALID_ARG;
+  int32_t* hist = permute_scratch_ptr();
+  unsigned* err = check_word_ptr();
+  if (!hist || !err) return STRATA_ERR_CUDA;
+  return cuda_status(launch_permute(topk_ids, dims.T, dims.k, dims.E, counts, offsets,
+                                    sorted_token, slot_row, hist, err, s));
+}
+
 strata_status_t strata_moe_expert_gemm_q4(strata_moe_op_t op, const uint16_t* a,
                                           const int32_t* sorted_token, const int32_t* offsets,
                                           strata_q4_t w0, strata_q4_t w1,

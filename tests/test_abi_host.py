@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert names == {
         "strata_moe_workspace_bytes", "strata_status_string", "strata_moe_route",
-        "strata_moe_permute", "strata_moe_expert_gemm_q4", "strata_moe_combine",
+        "strata_moe_permute", "strata_moe_permute_static", "strata_moe_expert_gemm_q4",
+        "strata_moe_combine",
         "strata_moe_forward", "strata_moe_device_status"}
 
 
