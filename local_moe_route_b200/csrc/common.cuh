@@ -287,6 +287,11 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
 // Warp helpers
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// Barrier `id` (1..15) among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

@@ -57,20 +57,20 @@ constexpr int BM = 128;                    // weight rows per slot (TMEM lanes)
 constexpr int NT = kTileRows;              // token rows per unit (max MMA N)
 constexpr int BK = 64;                     // K per stage
 constexpr int RAW_ST = 8;                  // packed-weight ring depth
-constexpr int B_ST = 6;                    // token-row ring depth
+constexpr int B_ST = 4;                    // token-row ring depth
 constexpr int A_ST = 4;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
-constexpr int EPI_PITCH = 40;              // halves per transpose-tile row (80 B)
+constexpr int STG_PITCH = 2 * BM + 8;      // halves per staging row (up to 256 outputs)
 
 constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3, W_EPI = 11;
 constexpr int THREADS = 15 * 32;
 
 constexpr int RAW_OFF = 0;                                        // [RAW_ST][2][RAW_BYTES]
 constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;           // [B_ST][B_BYTES]
-constexpr int EPI_OFF = B_OFF + B_ST * B_BYTES;                   // [4][32][EPI_PITCH] fp16
-constexpr int EPI_BYTES = 4 * 32 * EPI_PITCH * 2;
-constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
+constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;                   // [NT][STG_PITCH] fp16
+constexpr int STG_BYTES = NT * STG_PITCH * 2;
+constexpr int BAR_OFF = STG_OFF + STG_BYTES;
 constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
 constexpr int TOK_OFF = BAR_OFF + NBARS * 8;
 constexpr int MISC_OFF = TOK_OFF + NT * 4;
@@ -125,16 +125,22 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int u, int FB) {
   return U;
 }
 
-// 8 int4 (natural order: nibble i = element i) -> 4 fp16 pairs = RNE(q * s).
+// Packed int4 codes hold element i of a group of 8 in nibble i as a two's
+// complement value q in [-8, 7].  XOR with 0x8 turns a nibble into q + 8, and
+// placing q + 8 in the low mantissa bits of fp16 1024.0 gives 1032 + q
+// exactly; subtracting 1032 leaves q and one fp16 multiply gives the weight
+// RNE_fp16(q * s).
+
+// 8 codes -> 4 fp16 pairs in natural K order: pair i = (element 2i, 2i+1).
 __device__ __forceinline__ void dequant8(uint32_t w, uint32_t sc2, uint32_t* r) {
-  const uint32_t w4 = w >> 4;
+  const uint32_t wx = w ^ 0x88888888u;
+  const uint32_t wx4 = wx >> 4;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // byte i of w (element 2i in its low nibble) to the low half, byte i of
-    // w >> 4 (element 2i+1 in its low nibble) to the high half
-    const uint32_t t = __byte_perm(w, w4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
-    // fp16 pair 1024 + (nibble ^ 8) = 1032 + q
-    const uint32_t v = ((t ^ 0x64086408u) & 0x000F000Fu) | 0x64006400u;
+    // byte i of wx (element 2i in its low nibble) to the low half, byte i of
+    // wx >> 4 (element 2i+1 in its low nibble) to the high half
+    const uint32_t t = __byte_perm(wx, wx4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
+    const uint32_t v = (t & 0x000F000Fu) | 0x64006400u;        // 1032 + q, both halves
     uint32_t qv, o;
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(qv) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o) : "r"(qv), "r"(sc2));
@@ -142,9 +148,34 @@ __device__ __forceinline__ void dequant8(uint32_t w, uint32_t sc2, uint32_t* r) 
   }
 }
 
-// Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]) for the S grouped rows.
-// Out-of-range token indices are reported (kErrIndex) and read row 0; values
-// beyond the fp16 range become +-inf and are reported as kErrRange.
+// 8 codes -> 4 fp16 pairs in the interleaved K order (0,4), (1,5), (2,6),
+// (3,7): each pair comes out of one mask-and-or, with no byte permute.  The
+// operand it is multiplied with must use the same order within each group
+// of 8 (the grouped fp16 copy of x is written that way).
+__device__ __forceinline__ void dequant8_interleaved(uint32_t w, uint32_t sc2, uint32_t* r) {
+  const uint32_t wx = w ^ 0x88888888u;
+  const uint32_t wx8 = wx >> 8;
+  const uint32_t v0 = (wx & 0x000F000Fu) | 0x64006400u;   // 1024 + (q + 8):   elements 0, 4
+  const uint32_t v1 = (wx & 0x00F000F0u) | 0x64006400u;   // 1024 + 16(q + 8): elements 1, 5
+  const uint32_t v2 = (wx8 & 0x000F000Fu) | 0x64006400u;  // elements 2, 6
+  const uint32_t v3 = (wx8 & 0x00F000F0u) | 0x64006400u;  // elements 3, 7
+  uint32_t q0, q1, q2, q3;
+  // 1024 + (q + 8) - 1032 = q;  (1024 + 16(q + 8)) / 16 - 72 = q  (all exact)
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q0) : "r"(v0), "r"(0x3C003C00u), "r"(0xE408E408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q1) : "r"(v1), "r"(0x2C002C00u), "r"(0xD480D480u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q2) : "r"(v2), "r"(0x3C003C00u), "r"(0xE408E408u));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q3) : "r"(v3), "r"(0x2C002C00u), "r"(0xD480D480u));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(q0), "r"(sc2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[1]) : "r"(q1), "r"(sc2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(q2), "r"(sc2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[3]) : "r"(q3), "r"(sc2));
+}
+
+// Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]) for the S grouped rows,
+// with K interleaved within each group of 8 (0, 4, 1, 5, 2, 6, 3, 7) to match
+// dequant8_interleaved.  Out-of-range token indices are reported (kErrIndex)
+// and read row 0; values beyond the fp16 range become +-inf and are reported
+// as kErrRange.
 __global__ void __launch_bounds__(256)
     gather_rows_f16_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
                            int T, int d, int S, uint16_t* __restrict__ xs, unsigned* err) {
@@ -160,14 +191,17 @@ __global__ void __launch_bounds__(256)
       t = 0;
     }
     const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8);
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    float e[8];
+    e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
+    e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
+    // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
+    // weight dequantisation produces)
     uint32_t out[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = bf16_lo(in[j]), hi = bf16_hi(in[j]);
-      over |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-      out[j] = (uint32_t)f16_bits(lo) | ((uint32_t)f16_bits(hi) << 16);
-    }
+    for (int j = 0; j < 4; ++j)
+      out[j] = (uint32_t)f16_bits(e[j]) | ((uint32_t)f16_bits(e[j + 4]) << 16);
     *reinterpret_cast<uint4*>(xs + (size_t)p * d + c * 8) = make_uint4(out[0], out[1], out[2], out[3]);
   }
   if (over) atomicOr(err, kErrRange);
@@ -185,7 +219,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* sRaw = smem + RAW_OFF;
   uint8_t* sB = smem + B_OFF;
-  uint16_t* sEpi = reinterpret_cast<uint16_t*>(smem + EPI_OFF);
+  uint16_t* sStg = reinterpret_cast<uint16_t*>(smem + STG_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + RAW_ST;
@@ -370,7 +404,6 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * sw);
         raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * (sw ^ 1));
       }
-      mbar_arrive(&raw_empty[sr]);
       if (g >= A_ST && !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
         break;
       __syncwarp();       // converged before the .sync.aligned TMEM stores
@@ -383,25 +416,37 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                                    raw[m][1].x, raw[m][1].y, raw[m][1].z, raw[m][1].w};
         uint32_t out[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
+        for (int c = 0; c < 8; ++c) {
+          if (OP == 0) dequant8_interleaved(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
+          else dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
+        }
         tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
       }
+      // The packed words have been consumed (the dequantisation above used
+      // them), so the next TMA write into this raw stage cannot overtake a
+      // shared-memory load still in flight.
+      mbar_arrive(&raw_empty[sr]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&a_full[sa]);
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    // Accumulator -> fp16 staging tile [token][feature] in shared memory; the
+    // accumulator is handed back to the MMA warp as soon as it has been read,
+    // and the staging tile then goes to global memory with coalesced 16-byte
+    // stores while the next unit's MMAs run.
     const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int et = threadIdx.x - W_EPI * 32;          // 0..127
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
-    uint16_t* tile = sEpi + (warp - W_EPI) * 32 * EPI_PITCH;
     for (int i = 0; i < my_units; ++i) {
       const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
       if (!mbar_wait_warp(acc_full, i & 1, abort_flag, args.err)) break;
       tc_fence_after();
       const int nch = (U.cnt + 31) >> 5;
-      for (int m = 0; m < (OP == 0 ? 1 : U.nslots); ++m) {
+      const int nout = OP == 0 ? 1 : U.nslots;        // 128-feature slices of output
+      for (int m = 0; m < nout; ++m) {
+        uint16_t* col = sStg + m * BM + q * 32 + lane;
         for (int c = 0; c < nch; ++c) {
           __syncwarp();   // converged before the .sync.aligned TMEM loads
           uint32_t a0[32];
@@ -413,34 +458,31 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
-              tile[j * EPI_PITCH + lane] = f16_bits(gv / (1.0f + __expf(-gv)) * uv);
+              col[(c * 32 + j) * STG_PITCH] = f16_bits(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
             }
           } else {
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               float v = __uint_as_float(a0[j]);
-              const int p = U.p0 + c * 32 + j;
-              if (args.row_scale && c * 32 + j < U.cnt) v *= args.row_scale[p];
-              tile[j * EPI_PITCH + lane] = f16_bits(v);
+              const int t = c * 32 + j;
+              if (args.row_scale && t < U.cnt) v *= args.row_scale[U.p0 + t];
+              col[t * STG_PITCH] = f16_bits(v);
             }
           }
-          __syncwarp();
-          // thread `lane` writes token row c*32 + lane: this warp's 32 features
-          if (c * 32 + lane < U.cnt) {
-            const uint4* src = reinterpret_cast<const uint4*>(tile + lane * EPI_PITCH);
-            uint4* dst = reinterpret_cast<uint4*>(
-                args.out + (size_t)(U.p0 + c * 32 + lane) * N + U.fout[m] + q * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = src[v];
-          }
-          __syncwarp();
         }
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
+      named_barrier_sync(1, 128);                     // staging tile complete
+      const int cpr = nout * (BM / 8);                // 16-byte chunks per row
+      for (int idx = et; idx < U.cnt * cpr; idx += 128) {
+        const int row = idx / cpr, ch = idx - row * cpr;
+        const uint4 v = *reinterpret_cast<const uint4*>(sStg + row * STG_PITCH + ch * 8);
+        *reinterpret_cast<uint4*>(args.out + (size_t)(U.p0 + row) * N + U.fout[0] + ch * 8) = v;
+      }
+      named_barrier_sync(1, 128);                     // staging tile free again
     }
-    (void)r;
   }
 
   tc_fence_before();
