@@ -287,6 +287,15 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
 // Warp helpers
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// True in exactly one lane of the (fully converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p)::"memory");
+  return p != 0;
+}
+
 // Barrier `id` (1..15) among `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -318,24 +318,27 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     }
   } else if (warp == W_MMA) {
     // -------------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      uint32_t g = 0;
-      bool stop = false;
-      for (int i = 0; i < my_units && !stop; ++i) {
-        const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
-        const uint32_t idesc = idesc_f32acc(BM, U.nrows, kFmtF16, 0);
-        if (i > 0) {
-          if (!mbar_wait(acc_empty, (i - 1) & 1, abort_flag, args.err)) break;
-          tc_fence_after();
+    // The whole warp follows the rings; one lane, elected once, issues every
+    // MMA and commit (a commit covers the MMAs of the thread that issues it).
+    uint32_t g = 0;
+    bool stop = false;
+    const bool leader = elect_one();
+    for (int i = 0; i < my_units && !stop; ++i) {
+      const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
+      const uint32_t idesc = idesc_f32acc(BM, U.nrows, kFmtF16, 0);
+      if (i > 0) {
+        if (!mbar_wait_warp(acc_empty, (i - 1) & 1, abort_flag, args.err)) break;
+        tc_fence_after();
+      }
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        const int sa = g % A_ST, sb = g % B_ST;
+        if (!mbar_wait_warp(&a_full[sa], (g / A_ST) & 1, abort_flag, args.err) ||
+            !mbar_wait_warp(&b_full[sb], (g / B_ST) & 1, abort_flag, args.err)) {
+          stop = true;
+          break;
         }
-        for (int kb = 0; kb < KB; ++kb, ++g) {
-          const int sa = g % A_ST, sb = g % B_ST;
-          if (!mbar_wait(&a_full[sa], (g / A_ST) & 1, abort_flag, args.err) ||
-              !mbar_wait(&b_full[sb], (g / B_ST) & 1, abort_flag, args.err)) {
-            stop = true;
-            break;
-          }
-          tc_fence_after();
+        tc_fence_after();
+        if (leader) {
           const uint32_t b0 = smem_addr(sB + sb * B_BYTES);
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
@@ -350,10 +353,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           mma_commit(&a_empty[sa]);
           mma_commit(&b_empty[sb]);
         }
-        if (!stop) mma_commit(acc_full);
+        __syncwarp();
       }
+      if (!stop && leader) mma_commit(acc_full);
+      __syncwarp();
     }
-    __syncwarp();
   } else if (warp < W_EPI) {
     // -------------------------------------------------------------- dequantise
     const int wg = (warp - W_DQ) >> 2;       // takes the stages g with g % 2 == wg
