@@ -61,15 +61,15 @@ constexpr int B_ST = 4;                    // token-row ring depth
 constexpr int A_ST = 4;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
-constexpr int STG_PITCH = 2 * BM + 8;      // halves per staging row (up to 256 outputs)
+constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output feature)
 
 constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3, W_EPI = 11;
 constexpr int THREADS = 15 * 32;
 
 constexpr int RAW_OFF = 0;                                        // [RAW_ST][2][RAW_BYTES]
 constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;           // [B_ST][B_BYTES]
-constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;                   // [NT][STG_PITCH] fp16
-constexpr int STG_BYTES = NT * STG_PITCH * 2;
+constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;                   // [2 * BM][STG_PITCH] fp16
+constexpr int STG_BYTES = 2 * BM * STG_PITCH * 2;
 constexpr int BAR_OFF = STG_OFF + STG_BYTES;
 constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
 constexpr int TOK_OFF = BAR_OFF + NBARS * 8;
@@ -436,10 +436,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    // Accumulator -> fp16 staging tile [token][feature] in shared memory; the
-    // accumulator is handed back to the MMA warp as soon as it has been read,
-    // and the staging tile then goes to global memory with coalesced 16-byte
-    // stores while the next unit's MMAs run.
+    // The accumulator is read out in the layout TMEM holds it, one output
+    // feature per thread: its token values go as packed fp16 into a staging
+    // tile [feature][token] in shared memory (four 16-byte stores per 32
+    // tokens), and the accumulator is handed back to the MMA warp right
+    // after.  The transposition to the row-major output happens on the way
+    // out: thread t gathers 8 features of token t and stores 16 bytes, while
+    // the next unit's MMAs already run.
     const int q = warp & 3;
     const int et = threadIdx.x - W_EPI * 32;          // 0..127
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
@@ -450,11 +453,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const int nch = (U.cnt + 31) >> 5;
       const int nout = OP == 0 ? 1 : U.nslots;        // 128-feature slices of output
       for (int m = 0; m < nout; ++m) {
-        uint16_t* col = sStg + m * BM + q * 32 + lane;
+        uint16_t* frow = sStg + (m * BM + q * 32 + lane) * STG_PITCH;
         for (int c = 0; c < nch; ++c) {
           __syncwarp();   // converged before the .sync.aligned TMEM loads
           uint32_t a0[32];
           tmem_ld_32x32b_x32(t_lane + m * BM + c * 32, a0);
+          float v[32];
           if (OP == 0) {
             uint32_t a1[32];
             tmem_ld_32x32b_x32(t_lane + BM + c * 32, a1);
@@ -462,28 +466,48 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
-              col[(c * 32 + j) * STG_PITCH] = f16_bits(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+              v[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
             }
           } else {
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float v = __uint_as_float(a0[j]);
-              const int t = c * 32 + j;
-              if (args.row_scale && t < U.cnt) v *= args.row_scale[U.p0 + t];
-              col[t * STG_PITCH] = f16_bits(v);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a0[j]);
+            if (args.row_scale) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int t = c * 32 + j;
+                if (t < U.cnt) v[j] *= args.row_scale[U.p0 + t];
+              }
             }
+          }
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            uint4 o;
+            o.x = pack_f16x2(v[8 * k4 + 0], v[8 * k4 + 1]);
+            o.y = pack_f16x2(v[8 * k4 + 2], v[8 * k4 + 3]);
+            o.z = pack_f16x2(v[8 * k4 + 4], v[8 * k4 + 5]);
+            o.w = pack_f16x2(v[8 * k4 + 6], v[8 * k4 + 7]);
+            *reinterpret_cast<uint4*>(frow + c * 32 + 8 * k4) = o;
           }
         }
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
       named_barrier_sync(1, 128);                     // staging tile complete
-      const int cpr = nout * (BM / 8);                // 16-byte chunks per row
-      for (int idx = et; idx < U.cnt * cpr; idx += 128) {
-        const int row = idx / cpr, ch = idx - row * cpr;
-        const uint4 v = *reinterpret_cast<const uint4*>(sStg + row * STG_PITCH + ch * 8);
-        *reinterpret_cast<uint4*>(args.out + (size_t)(U.p0 + row) * N + U.fout[0] + ch * 8) = v;
+      if (et < U.cnt) {
+        uint16_t* dst = args.out + (size_t)(U.p0 + et) * N + U.fout[0];
+        for (int ch = 0; ch < nout * (BM / 8); ++ch) {
+          const uint16_t* src = sStg + ch * 8 * STG_PITCH + et;
+          uint32_t h[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) h[k] = src[k * STG_PITCH];
+          uint4 o;
+          o.x = __byte_perm(h[0], h[1], 0x5410);
+          o.y = __byte_perm(h[2], h[3], 0x5410);
+          o.z = __byte_perm(h[4], h[5], 0x5410);
+          o.w = __byte_perm(h[6], h[7], 0x5410);
+          *reinterpret_cast<uint4*>(dst + ch * 8) = o;
+        }
       }
       named_barrier_sync(1, 128);                     // staging tile free again
     }
