@@ -106,7 +106,7 @@ SchedRegions add_schedule(Layout& L, const strata_moe_dims_t& d) {
   const int S = d.T * d.k;
   SchedRegions r;
   r.tile_prefix = L.add((size_t)(d.E + 1) * sizeof(int32_t));
-  r.tile_table = L.add((size_t)max_tiles(S, d.E) * sizeof(int2));
+  r.tile_table = L.add((size_t)max_tiles(S, d.E) * sizeof(int4));
   r.active = L.add((size_t)d.E * sizeof(int32_t));
   r.n_active = L.add(sizeof(int32_t));
   return r;
@@ -114,7 +114,7 @@ SchedRegions add_schedule(Layout& L, const strata_moe_dims_t& d) {
 Schedule schedule_at(uint8_t* ws, const SchedRegions& r) {
   Schedule s;
   s.tile_prefix = reinterpret_cast<int32_t*>(ws + r.tile_prefix.off);
-  s.tile_table = reinterpret_cast<int2*>(ws + r.tile_table.off);
+  s.tile_table = reinterpret_cast<int4*>(ws + r.tile_table.off);
   s.active = reinterpret_cast<int32_t*>(ws + r.active.off);
   s.n_active = reinterpret_cast<int32_t*>(ws + r.n_active.off);
   return s;

@@ -84,7 +84,7 @@ struct TcArgs {
   const uint16_t* a;            // B operand rows (fp16): x16 [T][K] or h [S][K]
   const int32_t* sorted_token;  // gate/up: row -> token
   const int32_t* offsets;
-  const int2* tile_table;
+  const int4* tile_table;        // (expert, first row, rows, 0) per tile
   const int32_t* total_tiles;   // -> tile_prefix[E]
   const uint16_t* s0;
   const uint16_t* s1;
@@ -105,11 +105,11 @@ struct Unit {
 template <int OP>
 __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int u, int FB) {
   Unit U;
-  const int2 te = a.tile_table[u / FB];
+  const int4 te = a.tile_table[u / FB];
   const int fb = u % FB;
   U.e = te.x;
-  U.p0 = a.offsets[U.e] + te.y * tc::NT;
-  U.cnt = min(tc::NT, a.offsets[U.e + 1] - U.p0);
+  U.p0 = te.y;
+  U.cnt = te.z;
   U.nrows = (U.cnt + 15) & ~15;
   if (OP == 0) {
     U.nslots = 2;
@@ -365,38 +365,88 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int r = q * 32 + lane;             // weight row within the slot
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     const int g_shift = G == 32 ? 5 : (G == 64 ? 6 : 7);
-    int pf_i = -1;
-    Unit pf_U;
-    // Scales of stage gs for this row (both slots; with 32-wide groups the
-    // stage spans two groups): sc[m][0], sc[m][1] as fp16 bits.
-    auto load_scales = [&](int gs, uint32_t (&sc)[2][2]) {
-      if (gs >= total_stages) return;
-      const int i = gs / KB, kb = gs - i * KB;
-      if (i != pf_i) {
-        pf_U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
-        pf_i = i;
-      }
-      const int grp = (kb * BK) >> g_shift;
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint16_t* sp = (OP == 0 && m == 1) ? args.s1 : args.s0;
-        if (m < pf_U.nslots) {
-          const uint16_t* p = sp + (size_t)(pf_U.wrow[m] + r) * (K / G) + grp;
-          sc[m][0] = __ldg(p);
-          sc[m][1] = G == 32 ? __ldg(p + 1) : sc[m][0];
-        } else {
-          sc[m][0] = sc[m][1] = 0;
-        }
-      }
+    const int KG = K / G;                    // groups per weight row
+    // Group scales are read in blocks of SB consecutive groups per row and
+    // slot (SB = the largest of 8, 4, 2, 1 dividing K / G, so a block is one
+    // aligned 16-, 8-, 4- or 2-byte load).  The block after the one in use
+    // is always in flight: a load has the time of SB groups to arrive.
+    const int SB = (KG & 7) == 0 ? 8 : (KG & 3) == 0 ? 4 : (KG & 1) == 0 ? 2 : 1;
+    int4 te_c = make_int4(0, 0, 0, 0), te_n = make_int4(0, 0, 0, 0);
+    int unit_c = -1;
+    auto tile_of = [&](int i) { return args.tile_table[(blockIdx.x + i * gridDim.x) / FB]; };
+    // first scale of block b0, slot mm, of unit i (tile entry te)
+    auto scale_ptr = [&](const int4& te, int i, int mm, int b0) {
+      const int fb = (blockIdx.x + i * gridDim.x) % FB;
+      int f0 = OP == 0 ? fb * BM : fb * 2 * BM + mm * BM;
+      if (f0 >= N) f0 -= BM;                 // a down slot beyond N: its results are unused
+      const uint16_t* sp = (OP == 0 && mm == 1) ? args.s1 : args.s0;
+      return sp + (size_t)(te.x * N + f0 + r) * KG + b0;
     };
-    uint32_t sc_next[2][2] = {{0, 0}, {0, 0}};
-    load_scales(wg, sc_next);
+    auto load_block = [&](const uint16_t* p) -> uint4 {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (SB == 8) {
+        v = __ldg(reinterpret_cast<const uint4*>(p));
+      } else if (SB == 4) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+        v.x = t.x;
+        v.y = t.y;
+      } else if (SB == 2) {
+        v.x = __ldg(reinterpret_cast<const uint32_t*>(p));
+      } else {
+        v.x = __ldg(p);
+      }
+      return v;
+    };
+    auto scale_at = [&](const uint4& v, int idx) -> uint32_t {
+      const int w = idx >> 1;
+      const uint32_t x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+      return (idx & 1) ? (x >> 16) : (x & 0xFFFFu);
+    };
+    uint4 blk_c[2], blk_n[2];
+    int key_c = -1, key_n = -1;              // unit * 65536 + first group of the block
     for (int j = 0;; ++j) {
       const int g = wg + 2 * j;
       if (g >= total_stages) break;
-      // the loads of this stage's scales were issued a whole own stage ago
-      const uint32_t sc_cur[2][2] = {{sc_next[0][0], sc_next[0][1]}, {sc_next[1][0], sc_next[1][1]}};
-      load_scales(g + 2, sc_next);
+      const int iu = g / KB, kb = g - iu * KB;
+      const int grp0 = (kb * BK) >> g_shift;
+      const int key = (iu << 16) | (grp0 & ~(SB - 1));
+      if (key != key_c) {
+        if (iu != unit_c) {
+          te_c = (unit_c >= 0 && iu == unit_c + 1) ? te_n : tile_of(iu);
+          unit_c = iu;
+          if (iu + 1 < my_units) te_n = tile_of(iu + 1);
+        }
+        if (key == key_n) {
+          blk_c[0] = blk_n[0];
+          blk_c[1] = blk_n[1];
+        } else {
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+            blk_c[mm] = load_block(scale_ptr(te_c, iu, mm, key & 0xFFFF));
+        }
+        key_c = key;
+        // the block after this one: the next groups of this unit, or the
+        // first block of the next unit
+        int ni = iu, nb = (key & 0xFFFF) + SB;
+        if (nb >= KG) {
+          nb = 0;
+          ++ni;
+        }
+        key_n = -1;
+        if (ni < my_units) {
+          key_n = (ni << 16) | nb;
+#pragma unroll
+          for (int mm = 0; mm < 2; ++mm)
+            blk_n[mm] = load_block(scale_ptr(ni == iu ? te_c : te_n, ni, mm, nb));
+        }
+      }
+      const int idx = grp0 & (SB - 1);
+      uint32_t sc_cur[2][2];
+#pragma unroll
+      for (int mm = 0; mm < 2; ++mm) {
+        sc_cur[mm][0] = scale_at(blk_c[mm], idx);
+        sc_cur[mm][1] = G == 32 ? scale_at(blk_c[mm], idx + 1) : sc_cur[mm][0];
+      }
       const int sr = g % RAW_ST, sa = g % A_ST;
       if (!mbar_wait(&raw_full[sr], (g / RAW_ST) & 1, abort_flag, args.err)) break;
       // packed words of this row; 32-byte swizzle puts chunk c at c ^ ((r >> 2) & 1)

@@ -19,7 +19,7 @@ constexpr int kStreamMaxTokens = 8;
 // Per-expert work lists derived from offsets (built on the device).
 struct Schedule {
   int32_t* tile_prefix;   // [E+1]  tiles of kTileRows rows before expert e; [E] = total
-  int2* tile_table;       // [max_tiles] (expert, tile index within the expert)
+  int4* tile_table;       // [max_tiles] (expert, first grouped row, rows, 0)
   int32_t* active;        // [E]   experts with at least one row, ascending
   int32_t* n_active;      // [1]
 };

@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(1024)
   const int ap = block_exclusive_scan(cnt > 0 ? 1 : 0, &total_active);
   if (e < E) {
     sch.tile_prefix[e] = tp;
-    for (int j = 0; j < tiles; ++j) sch.tile_table[tp + j] = make_int2(e, j);
+    for (int j = 0; j < tiles; ++j) {
+      const int p0 = offsets[e] + j * kTileRows;
+      sch.tile_table[tp + j] = make_int4(e, p0, min(kTileRows, cnt - j * kTileRows), 0);
+    }
     if (cnt > 0) sch.active[ap] = e;
   }
   if (e == 0) {
