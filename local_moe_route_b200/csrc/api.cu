@@ -175,7 +175,8 @@ strata_status_t do_route(const uint16_t* x, const uint16_t* w_router, const floa
 strata_status_t do_gemm(int op, const uint16_t* a, const int32_t* sorted_token,
                         const int32_t* offsets, strata_q4_t w0, strata_q4_t w1,
                         const float* row_scale, const strata_moe_dims_t& d, uint16_t* out,
-                        const Schedule& sch, uint16_t* x16, unsigned* err, cudaStream_t s) {
+                        const Schedule& sch, uint16_t* x16, unsigned* err, cudaStream_t s,
+                        bool h_interleaved = false) {
   GemmProblem p;
   p.op = op;
   p.a = a;
@@ -195,6 +196,7 @@ strata_status_t do_gemm(int op, const uint16_t* a, const int32_t* sorted_token,
   p.N = op == 0 ? d.n : d.d;
   p.G = d.group;
   p.err = err;
+  p.h_interleaved = h_interleaved;
   const cudaError_t e = d.T <= kStreamMaxTokens ? launch_gemm_stream(p, sch, s)
                                                 : launch_gemm_tc(p, sch, s);
   return cuda_status(e);
@@ -394,10 +396,12 @@ strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router, 
   if (launch_schedule(offsets, dims.E, dims.T * dims.k, sch, err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
   uint16_t* x16 = reinterpret_cast<uint16_t*>(at(f.x16));
-  st = do_gemm(0, x, sorted_token, offsets, gate, up, nullptr, dims, h, sch, x16, err, s);
+  // h is internal here: it passes between the GEMMs in the interleaved
+  // feature order the down projection's dequantisation produces
+  st = do_gemm(0, x, sorted_token, offsets, gate, up, nullptr, dims, h, sch, x16, err, s, true);
   if (st != STRATA_OK) return st;
   const strata_q4_t none = {nullptr, nullptr};
-  st = do_gemm(1, h, nullptr, offsets, down, none, nullptr, dims, rows, sch, x16, err, s);
+  st = do_gemm(1, h, nullptr, offsets, down, none, nullptr, dims, rows, sch, x16, err, s, true);
   if (st != STRATA_OK) return st;
   return cuda_status(launch_combine_checked(rows, w, slot_row, dims.T, dims.k, dims.d, y, err, s));
 }

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(256)
   if (bad) atomicOr(err, kErrIndex);
 }
 
-template <int OP>
+template <int OP, bool ILV>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
                           const __grid_constant__ CUtensorMap map_q1,
@@ -397,17 +397,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       }
       return v;
     };
-    auto scale_at = [&](const uint4& v, int idx) -> uint32_t {
-      const int w = idx >> 1;
-      const uint32_t x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
-      return (idx & 1) ? (x >> 16) : (x & 0xFFFFu);
+    // the 32-bit word of a block holding groups 2w and 2w + 1
+    auto word_at = [&](const uint4& v, int w) -> uint32_t {
+      return (w & 2) ? ((w & 1) ? v.w : v.z) : ((w & 1) ? v.y : v.x);
     };
     uint4 blk_c[2], blk_n[2];
     int key_c = -1, key_n = -1;              // unit * 65536 + first group of the block
-    for (int j = 0;; ++j) {
-      const int g = wg + 2 * j;
-      if (g >= total_stages) break;
-      const int iu = g / KB, kb = g - iu * KB;
+    int iu = 0, kb = wg;                     // unit and K block of stage g (KB >= 2)
+    for (int g = wg; g < total_stages; g += 2) {
       const int grp0 = (kb * BK) >> g_shift;
       const int key = (iu << 16) | (grp0 & ~(SB - 1));
       if (key != key_c) {
@@ -440,12 +437,21 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             blk_n[mm] = load_block(scale_ptr(ni == iu ? te_c : te_n, ni, mm, nb));
         }
       }
+      // fp16 scale pairs (the scale in both halves) for the stage's group(s);
+      // with 32-wide groups the stage's two groups share one 32-bit word
       const int idx = grp0 & (SB - 1);
-      uint32_t sc_cur[2][2];
+      const uint32_t sel = (G != 32 && (idx & 1)) ? 0x3232u : 0x1010u;
+      uint32_t sc2[2][2];
 #pragma unroll
       for (int mm = 0; mm < 2; ++mm) {
-        sc_cur[mm][0] = scale_at(blk_c[mm], idx);
-        sc_cur[mm][1] = G == 32 ? scale_at(blk_c[mm], idx + 1) : sc_cur[mm][0];
+        const uint32_t w = word_at(blk_c[mm], idx >> 1);
+        sc2[mm][0] = __byte_perm(w, 0, sel);
+        sc2[mm][1] = G == 32 ? __byte_perm(w, 0, 0x3232u) : sc2[mm][0];
+      }
+      kb += 2;
+      if (kb >= KB) {
+        kb -= KB;
+        ++iu;
       }
       const int sr = g % RAW_ST, sa = g % A_ST;
       if (!mbar_wait(&raw_full[sr], (g / RAW_ST) & 1, abort_flag, args.err)) break;
@@ -464,14 +470,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
-        const uint32_t sc_a = sc_cur[m][0] | (sc_cur[m][0] << 16);
-        const uint32_t sc_b = sc_cur[m][1] | (sc_cur[m][1] << 16);
+        const uint32_t sc_a = sc2[m][0], sc_b = sc2[m][1];
         const uint32_t words[8] = {raw[m][0].x, raw[m][0].y, raw[m][0].z, raw[m][0].w,
                                    raw[m][1].x, raw[m][1].y, raw[m][1].z, raw[m][1].w};
         uint32_t out[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          if (OP == 0) dequant8_interleaved(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
+          // gate/up: the grouped copy of x is interleaved; down: h is
+          // interleaved when the fused forward produced it
+          if (OP == 0 || ILV) dequant8_interleaved(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
           else dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
         }
         tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
@@ -552,10 +559,17 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < 8; ++k) h[k] = src[k * STG_PITCH];
           uint4 o;
-          o.x = __byte_perm(h[0], h[1], 0x5410);
-          o.y = __byte_perm(h[2], h[3], 0x5410);
-          o.z = __byte_perm(h[4], h[5], 0x5410);
-          o.w = __byte_perm(h[6], h[7], 0x5410);
+          if (OP == 0 && ILV) {      // features 0,4 | 1,5 | 2,6 | 3,7 (see GemmProblem)
+            o.x = __byte_perm(h[0], h[4], 0x5410);
+            o.y = __byte_perm(h[1], h[5], 0x5410);
+            o.z = __byte_perm(h[2], h[6], 0x5410);
+            o.w = __byte_perm(h[3], h[7], 0x5410);
+          } else {
+            o.x = __byte_perm(h[0], h[1], 0x5410);
+            o.y = __byte_perm(h[2], h[3], 0x5410);
+            o.z = __byte_perm(h[4], h[5], 0x5410);
+            o.w = __byte_perm(h[6], h[7], 0x5410);
+          }
           *reinterpret_cast<uint4*>(dst + ch * 8) = o;
         }
       }
@@ -573,7 +587,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 
 static int g_num_sms = 0;
 
-template <int OP>
+template <int OP, bool ILV>
 static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
   CUtensorMap m0, m1;
   const uint64_t rows = (uint64_t)p.E * p.N;
@@ -595,7 +609,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP>,
+    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP, ILV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM);
     if (e != cudaSuccess) return e;
   }
@@ -632,12 +646,14 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < g_num_sms ? max_units : g_num_sms);
-  moe_gemm_q4_tc_kernel<OP><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
+  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
-  return p.op == 0 ? launch_tc_impl<0>(p, sch, s) : launch_tc_impl<1>(p, sch, s);
+  if (p.op == 0)
+    return p.h_interleaved ? launch_tc_impl<0, true>(p, sch, s) : launch_tc_impl<0, false>(p, sch, s);
+  return p.h_interleaved ? launch_tc_impl<1, true>(p, sch, s) : launch_tc_impl<1, false>(p, sch, s);
 }
 
 }  // namespace strata

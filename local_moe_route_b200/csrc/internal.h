@@ -64,6 +64,11 @@ struct GemmProblem {
   uint16_t* a16;                // scratch [T*k][d]: fp16 x rows in grouped order (TC gate/up)
   uint16_t* out;
   int T, S, E, K, N, G;         // K reduction dim, N output features
+  // Tensor-core path only, set by the fused forward: h travels between the
+  // two GEMMs with its features interleaved within groups of 8 (0,4,1,5,
+  // 2,6,3,7), the order the down projection's weight dequantisation
+  // produces: gate/up writes it that way, down reads it that way.
+  bool h_interleaved = false;
   unsigned* err;
 };
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
