@@ -114,6 +114,9 @@ def device_layer(inp, dev):
 def launches_per_step(T, d, E):
     """Kernel launches of one strata_moe_forward (mirrors the dispatch rules)."""
     n = 2                    # router logits + top-k/softmax
+    tc_router = T >= 128 and E % 128 == 0
+    if not tc_router and T <= 16 and d // 32 > 1:
+        n += 1               # sum of the K-split partial logits
     n += 3                   # permutation: histogram, scan, scatter
     n += 1                   # expert work lists
     n += 2 if T > 8 else 1   # gate/up (+ fp16 copy of x on the tensor-core path)
@@ -201,9 +204,24 @@ def run_ours(args, wl):
     def forward(x=None, out=None):
         st = sm.strata_moe_forward(L["x"] if x is None else x, L["w_router"], L["bias"], gate, up,
                                    down, dims, y if out is None else out, None, None, ws,
-                                   stream=stream)
+                                   stream=torch.cuda.current_stream())
         if st != sm.STRATA_OK:
             raise sm.StrataError(st, "forward")
+
+    # Small batches (decode / verify) replay the forward as one CUDA graph:
+    # ten short kernels would otherwise wait on host launch overhead.  Large
+    # batches launch eagerly (the GPU is the bottleneck there).
+    graph = None
+    if T <= 64:
+        forward()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            forward()
+        torch.cuda.synchronize()
+    step = graph.replay if graph is not None else forward
+    # weights a small batch touches can fit in L2; those runs flush it
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if T <= 64 else None
 
     def barrier():
         torch.cuda.synchronize()
@@ -213,23 +231,37 @@ def run_ours(args, wl):
 
     # ---- headline: K forwards, device time
     for _ in range(args.warmup):
-        forward()
+        step()
     clocks = ClockSampler(dev.index) if rank == 0 else None
     barrier()
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    ev0.record(stream)
-    step_ev[0].record(stream)
-    for i in range(args.steps):
-        forward()
-        step_ev[i + 1].record(stream)
-    ev1.record(stream)
-    barrier()
-    total_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
-    step_ms = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
+    if flush is None:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev0.record(stream)
+        step_ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            step_ev[i + 1].record(stream)
+        ev1.record(stream)
+        barrier()
+        step_ms = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
+        total_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    else:
+        # the touched weights would stay in L2 from one step to the next:
+        # overwrite L2 between steps and time each step alone
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a_, b_ in pairs:
+            flush.zero_()
+            a_.record(stream)
+            step()
+            b_.record(stream)
+        barrier()
+        step_ms = [a_.elapsed_time(b_) for a_, b_ in pairs]
+        total_ms = max_over_ranks(sum(step_ms), dev)
     clk = clocks.stop() if clocks else None
     assert sm.strata_moe_device_status(stream) == sm.STRATA_OK
 
@@ -335,6 +367,16 @@ def run_ours(args, wl):
                 "algorithmic_per_launch": bytes_,
                 "traffic": profiled_traffic("gemm_gate_up_" + wl.name)}
     layer_flops = 2.0 * S * 3 * d * n + 2.0 * T * d * E
+    layer_roof = None
+    if not tensor_bound:
+        # the whole layer against HBM: weights of the experts the batch touches,
+        # the router matrix, x and y, over the step time
+        per_exp = 3 * n * d // 2 + 3 * n * (d // wl.group) * 2
+        lbytes = touched * per_exp + d * E * 2 + 2 * T * d * 2
+        lach = lbytes / (ms_step / 1e3) / 1e9
+        layer_roof = {"bound": "hbm", "achieved": round(lach, 1), "peak": hbm, "unit": "GB/s",
+                      "frac": round(lach / hbm, 4), "bytes_per_step": lbytes,
+                      "experts_touched": touched}
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -342,13 +384,17 @@ def run_ours(args, wl):
         "data": "synthetic (seeded, shapes of the pages' workload)",
         "config": {"workload": wl.name, "T": T, "d": d, "E": E, "k": k, "n": n,
                    "group": wl.group, "router_bias": wl.zipf > 0,
-                   "l2": "inputs larger than L2 (3.4 GB of weights), no flush",
+                   "l2": ("L2 flushed between steps (256 MB write), each step timed alone"
+                          if flush is not None else
+                          "inputs larger than L2 (3.4 GB of weights), no flush"),
+                   "launch": "one CUDA graph per forward" if graph is not None else "eager",
                    "parallelism": f"replicas x{world}"},
         "layer_tflops": round(layer_flops / (ms_step / 1e3) / 1e12, 1),
         "step_ms": {"min": round(min(step_ms), 4), "median": round(statistics.median(step_ms), 4),
                     "max": round(max(step_ms), 4)},
         "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
         "roofline": roof,
+        "layer_roofline": layer_roof,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
         "gpu_launches": launches_per_step(T, d, E) * args.steps,

@@ -169,7 +169,8 @@ strata_status_t do_route(const uint16_t* x, const uint16_t* w_router, const floa
   else
     e = launch_router_logits_simt(x, w_router, d.T, d.d, d.E, ks, partial, s);
   if (e != cudaSuccess) return STRATA_ERR_CUDA;
-  return cuda_status(launch_topk_softmax(partial, ks, bias, d.T, d.E, d.k, ids, w, logits_out, s));
+  // either path leaves the logits in split 0 of `partial`
+  return cuda_status(launch_topk_softmax(partial, 1, bias, d.T, d.E, d.k, ids, w, logits_out, s));
 }
 
 strata_status_t do_gemm(int op, const uint16_t* a, const int32_t* sorted_token,

@@ -29,17 +29,18 @@ constexpr int THREADS = WARPS * 32;
 constexpr int UNROLL = 4;          // 64-K blocks whose loads are in flight together
 }  // namespace st
 
-// Exact integer pair (q_i, q_{i+4}) from nibbles i and i+4 of w, as bf16x2
-// (F16 = false: 136 + q in the mantissa of 128.0) or fp16x2 (F16 = true:
-// 1032 + q in the mantissa of 1024.0), then the exact subtraction.
+// Exact integer pair (q_i, q_{i+4}) from nibbles i and i+4 of a word whose
+// nibbles were XORed with 8 (wx = w ^ 0x88888888, so a nibble holds q + 8):
+// the nibble goes into the low mantissa bits of 128.0 (bf16, F16 = false) or
+// 1024.0 (fp16, F16 = true) and one exact fma subtracts 136 or 1032.
 template <bool F16>
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int i) {
+__device__ __forceinline__ uint32_t nib_pair(uint32_t wx, int i) {
   uint32_t q;
   if (F16) {
-    const uint32_t v = (((w >> (4 * i)) ^ 0x64086408u) & 0x000F000Fu) | 0x64006400u;
+    const uint32_t v = ((wx >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
   } else {
-    const uint32_t v = (((w >> (4 * i)) ^ 0x43084308u) & 0x000F000Fu) | 0x43004300u;
+    const uint32_t v = ((wx >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
     asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
   }
   return q;
@@ -74,6 +75,7 @@ struct StreamArgs {
   const float* row_scale;
   uint16_t* out;
   int K, N, G;
+  int kspl;                     // warps per unit (1, 2, 4 or 8), splitting K
   unsigned* err;
 };
 
@@ -84,6 +86,8 @@ __device__ __forceinline__ void half_block(float (&acc)[4], uint32_t wg, uint32_
                                            float sg, float sg8, uint32_t b00, uint32_t b01,
                                            uint32_t b10, uint32_t b11) {
   float c[4] = {0.f, 0.f, 0.f, 0.f};
+  wg ^= 0x88888888u;
+  wg8 ^= 0x88888888u;
   mma16816<F16>(c, nib_pair<F16>(wg, 0), nib_pair<F16>(wg8, 0), nib_pair<F16>(wg, 1),
                 nib_pair<F16>(wg8, 1), b00, b01);
   mma16816<F16>(c, nib_pair<F16>(wg, 2), nib_pair<F16>(wg8, 2), nib_pair<F16>(wg, 3),
@@ -95,7 +99,7 @@ __device__ __forceinline__ void half_block(float (&acc)[4], uint32_t wg, uint32_
 }
 
 template <int NMAT>
-__global__ void __launch_bounds__(st::THREADS)
+__global__ void __launch_bounds__(st::THREADS, 2)
     moe_gemm_q4_stream_kernel(const StreamArgs args) {
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;           // fragment row group / B column
@@ -104,10 +108,19 @@ __global__ void __launch_bounds__(st::THREADS)
   const int KB = K / 64;
   const int FG = N / 16;
   const int units = (*args.n_active) * FG;
-  const int gw = blockIdx.x * st::WARPS + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * st::WARPS;
+  const int warp = threadIdx.x >> 5;
+  // kspl warps share a unit, splitting K: the split sp covers 64-K blocks
+  // [kb_lo, kb_hi).  A block holds WARPS / kspl units side by side; the warps
+  // of one unit meet at their own named barrier.
+  const int kspl = args.kspl;
+  const int per_block = st::WARPS / kspl;
+  const int slot = warp / kspl, sp = warp - slot * kspl;
+  const int kb_lo = sp * KB / kspl, kb_hi = (sp + 1) * KB / kspl;
+  __shared__ float red[st::WARPS][32][8];
 
-  for (int u = gw; u < units; u += nwarps) {
+  for (int ub = blockIdx.x * per_block; ub < units; ub += gridDim.x * per_block) {
+    const int u = ub + slot;
+    if (u >= units) continue;            // the unit's warps skip together
     const int e = args.active[u / FG];
     const int f0 = (u % FG) * 16;
     const int p_begin = args.offsets[e];
@@ -139,13 +152,16 @@ __global__ void __launch_bounds__(st::THREADS)
       float acc1[4] = {0.f, 0.f, 0.f, 0.f};
 
       __syncwarp();   // mma.sync.aligned needs the warp converged
-      for (int kb0 = 0; kb0 < KB; kb0 += st::UNROLL) {
+      for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += st::UNROLL) {
         uint32_t wa[st::UNROLL][2][2], wb[st::UNROLL][2][2];   // [blk][half][row g / g+8]
         uint4 xa[st::UNROLL][2];
+        // group scales of rows g, g + 8 (gate, up) for each half-block, loaded
+        // with the weights so their latency overlaps the weight loads
+        uint16_t sa[st::UNROLL][2][2], sb[st::UNROLL][2][2];
 #pragma unroll
         for (int j = 0; j < st::UNROLL; ++j) {
           const int kb = kb0 + j;
-          if (kb < KB) {
+          if (kb < kb_hi) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int byte = kb * 32 + h * 16 + t * 4;
@@ -157,49 +173,78 @@ __global__ void __launch_bounds__(st::THREADS)
               }
               xa[j][h] = col_ok ? __ldg(reinterpret_cast<const uint4*>(brow + kb * 64 + h * 32 + t * 8))
                                 : make_uint4(0, 0, 0, 0);
+              const int grp = (kb * 64 + h * 32) / G;
+              sa[j][h][0] = __ldg(sg0 + grp);
+              sa[j][h][1] = __ldg(sg0b + grp);
+              if (NMAT == 2) {
+                sb[j][h][0] = __ldg(sg1 + grp);
+                sb[j][h][1] = __ldg(sg1b + grp);
+              }
             }
           }
         }
 #pragma unroll
         for (int j = 0; j < st::UNROLL; ++j) {
           const int kb = kb0 + j;
-          if (kb < KB) {
+          if (kb < kb_hi) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int grp = (kb * 64 + h * 32) / G;
               const uint4 x = xa[j][h];
               // B fragments: K slots (2t, 2t+1) <- elements (i, i+4), (2t+8, 2t+9) <- (i+1, i+5)
               const uint32_t b00 = __byte_perm(x.x, x.z, 0x5410);   // (0, 4)
               const uint32_t b01 = __byte_perm(x.x, x.z, 0x7632);   // (1, 5)
               const uint32_t b10 = __byte_perm(x.y, x.w, 0x5410);   // (2, 6)
               const uint32_t b11 = __byte_perm(x.y, x.w, 0x7632);   // (3, 7)
-              half_block<NMAT == 1>(acc0, wa[j][h][0], wa[j][h][1], __half2float(__ushort_as_half(__ldg(sg0 + grp))),
-                         __half2float(__ushort_as_half(__ldg(sg0b + grp))), b00, b01, b10, b11);
+              half_block<NMAT == 1>(acc0, wa[j][h][0], wa[j][h][1],
+                                    __half2float(__ushort_as_half(sa[j][h][0])),
+                                    __half2float(__ushort_as_half(sa[j][h][1])), b00, b01, b10, b11);
               if (NMAT == 2)
                 half_block<false>(acc1, wb[j][h][0], wb[j][h][1],
-                           __half2float(__ushort_as_half(__ldg(sg1 + grp))),
-                           __half2float(__ushort_as_half(__ldg(sg1b + grp))), b00, b01, b10, b11);
+                                  __half2float(__ushort_as_half(sb[j][h][0])),
+                                  __half2float(__ushort_as_half(sb[j][h][1])), b00, b01, b10, b11);
             }
           }
         }
       }
-      // C fragment: (row g, cols 2t, 2t+1), (row g+8, cols 2t, 2t+1)
+      // K-split partial sums: added in split order (the result does not
+      // depend on timing), then the first warp of the unit finishes the tile.
+      if (kspl > 1) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = c0 + 2 * t + (i & 1);
-        const int feat = f0 + g + (i >> 1) * 8;
-        if (col < cnt) {
-          float v;
-          if (NMAT == 2) {
-            const float gv = acc0[i], uv = acc1[i];
-            v = gv / (1.0f + __expf(-gv)) * uv;
-          } else {
-            v = acc0[i];
-            if (args.row_scale) v *= args.row_scale[p_begin + col];
+        for (int i = 0; i < 4; ++i) {
+          red[warp][lane][i] = acc0[i];
+          red[warp][lane][4 + i] = acc1[i];
+        }
+        named_barrier_sync(1 + slot, kspl * 32);
+        if (sp == 0) {
+          for (int w = 1; w < kspl; ++w) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc0[i] += red[warp + w][lane][i];
+              acc1[i] += red[warp + w][lane][4 + i];
+            }
           }
-          args.out[(size_t)(p_begin + col) * N + feat] = f16_bits(v);
         }
       }
+      if (sp == 0) {
+        // C fragment: (row g, cols 2t, 2t+1), (row g+8, cols 2t, 2t+1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = c0 + 2 * t + (i & 1);
+          const int feat = f0 + g + (i >> 1) * 8;
+          if (col < cnt) {
+            float v;
+            if (NMAT == 2) {
+              const float gv = acc0[i], uv = acc1[i];
+              v = gv / (1.0f + __expf(-gv)) * uv;
+            } else {
+              v = acc0[i];
+              if (args.row_scale) v *= args.row_scale[p_begin + col];
+            }
+            args.out[(size_t)(p_begin + col) * N + feat] = f16_bits(v);
+          }
+        }
+      }
+      if (kspl > 1) named_barrier_sync(1 + slot, kspl * 32);   // red is reused next tile
     }
   }
 }
@@ -231,8 +276,16 @@ cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaSt
   a.err = p.err;
   const int max_active = p.S < p.E ? p.S : p.E;
   const long units = (long)max_active * (p.N / 16);
-  long blocks = (units + st::WARPS - 1) / st::WARPS;
-  if (blocks > 4L * num_sms) blocks = 4L * num_sms;
+  // Enough warps in flight to cover HBM latency: about two unit-warps per
+  // resident warp slot (2 blocks of 8 warps per SM); fewer units -> more
+  // warps per unit, each taking a slice of K.
+  const int KB = p.K / 64;
+  int kspl = 1;
+  while (kspl < st::WARPS && kspl * 2 <= KB && units * kspl < 2L * num_sms * 16) kspl *= 2;
+  a.kspl = kspl;
+  const long per_block = st::WARPS / kspl;
+  long blocks = (units + per_block - 1) / per_block;
+  if (blocks > 2L * num_sms) blocks = 2L * num_sms;
   if (blocks < 1) blocks = 1;
   if (p.op == 0)
     moe_gemm_q4_stream_kernel<2><<<(int)blocks, st::THREADS, 0, s>>>(a);

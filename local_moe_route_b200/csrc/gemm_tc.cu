@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int SB = (KG & 7) == 0 ? 8 : (KG & 3) == 0 ? 4 : (KG & 1) == 0 ? 2 : 1;
     int4 te_c = make_int4(0, 0, 0, 0), te_n = make_int4(0, 0, 0, 0);
     int unit_c = -1;
-    auto tile_of = [&](int i) { return args.tile_table[(blockIdx.x + i * gridDim.x) / FB]; };
+    auto tile_of = [&](int i) { return ld_nc_s4(args.tile_table + (blockIdx.x + i * gridDim.x) / FB); };
     // first scale of block b0, slot mm, of unit i (tile entry te)
     auto scale_ptr = [&](const int4& te, int i, int mm, int b0) {
       const int fb = (blockIdx.x + i * gridDim.x) % FB;
@@ -385,15 +385,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     auto load_block = [&](const uint16_t* p) -> uint4 {
       uint4 v = make_uint4(0, 0, 0, 0);
       if (SB == 8) {
-        v = __ldg(reinterpret_cast<const uint4*>(p));
+        v = ld_nc_v4(p);
       } else if (SB == 4) {
-        const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+        const uint2 t = ld_nc_v2(p);
         v.x = t.x;
         v.y = t.y;
       } else if (SB == 2) {
-        v.x = __ldg(reinterpret_cast<const uint32_t*>(p));
+        v.x = ld_nc_u32(p);
       } else {
-        v.x = __ldg(p);
+        v.x = ld_nc_u16(p);
       }
       return v;
     };

@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(rs::THREADS)
       }
       __syncthreads();
       if (e0 < E) {
+#pragma unroll 8
         for (int i = 0; i < len; ++i) {
           const size_t off = (size_t)(kc + i) * E + e0;
           float w0, w1;
@@ -235,11 +236,39 @@ __global__ void __launch_bounds__(rs::THREADS)
   }
 }
 
+// Sums the K-split partial logits of (token blockIdx.y, experts blockIdx.x *
+// 32 ..) into split 0: warp j adds splits j, j + 8, ... and the eight warp
+// sums are added in warp order, so the result does not depend on timing.
+__global__ void __launch_bounds__(256)
+    router_split_reduce_kernel(float* __restrict__ partial, int ksplit, int T, int E) {
+  __shared__ float red[8][33];
+  const int el = threadIdx.x & 31, sg = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + el, t = blockIdx.y;
+  float acc = 0.f;
+  if (e < E) {
+#pragma unroll 4
+    for (int sp = sg; sp < ksplit; sp += 8) acc += partial[((size_t)sp * T + t) * E + e];
+  }
+  red[sg][el] = acc;
+  __syncthreads();
+  if (sg == 0 && e < E) {
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sum += red[j][el];
+    partial[(size_t)t * E + e] = sum;
+  }
+}
+
+// Logits into split 0 of `partial` (the other splits are scratch).
 cudaError_t launch_router_logits_simt(const uint16_t* x, const uint16_t* w_router, int T, int d,
                                       int E, int ksplit, float* partial, cudaStream_t s) {
   const int rows = (d + ksplit - 1) / ksplit;
   dim3 grid((E + rs::EXPERTS - 1) / rs::EXPERTS, ksplit);
   router_logits_simt_kernel<<<grid, rs::THREADS, 0, s>>>(x, w_router, T, d, E, rows, partial);
+  if (ksplit > 1) {
+    dim3 rgrid((E + 31) / 32, T);
+    router_split_reduce_kernel<<<rgrid, 256, 0, s>>>(partial, ksplit, T, E);
+  }
   return cudaGetLastError();
 }
 
