@@ -179,30 +179,35 @@ __device__ __forceinline__ void dequant8_interleaved(uint32_t w, uint32_t sc2, u
 __global__ void __launch_bounds__(256)
     gather_rows_f16_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
                            int T, int d, int S, uint16_t* __restrict__ xs, unsigned* err) {
+  // one warp per grouped row; lane l converts 16-byte chunks l, l + 32, ...
+  const int lane = threadIdx.x & 31;
   const int cpr = d / 8;                      // 16-byte chunks per row
-  const size_t n = (size_t)S * cpr;
   bool over = false, bad = false;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const int p = (int)(i / cpr), c = (int)(i - (size_t)p * cpr);
+  for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < S; p += gridDim.x * 8) {
     int t = sorted_token[p];
     if ((unsigned)t >= (unsigned)T) {
       bad = true;
       t = 0;
     }
-    const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)t * d + c * 8);
-    float e[8];
-    e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
-    e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * d);
+#pragma unroll 2
+    for (int c = lane; c < cpr; c += 32) {
+      const uint4 v = __ldg(src + c);
+      float e[8];
+      e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
+      e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
-    // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
-    // weight dequantisation produces)
-    uint32_t out[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      out[j] = (uint32_t)f16_bits(e[j]) | ((uint32_t)f16_bits(e[j + 4]) << 16);
-    *reinterpret_cast<uint4*>(xs + (size_t)p * d + c * 8) = make_uint4(out[0], out[1], out[2], out[3]);
+      for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
+      // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
+      // weight dequantisation produces)
+      uint4 o;
+      o.x = pack_f16x2(e[0], e[4]);
+      o.y = pack_f16x2(e[1], e[5]);
+      o.z = pack_f16x2(e[2], e[6]);
+      o.w = pack_f16x2(e[3], e[7]);
+      dst[c] = o;
+    }
   }
   if (over) atomicOr(err, kErrRange);
   if (bad) atomicOr(err, kErrIndex);
@@ -621,8 +626,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   }
   if (OP == 0) {
     // the gate/up B operand: fp16 rows of x in grouped order
-    const size_t n = (size_t)p.S * (p.K / 8);
-    long blocks = (long)((n + 255) / 256);
+    long blocks = (p.S + 7) / 8;                     // 8 rows (warps) per block
     if (blocks > 16L * g_num_sms) blocks = 16L * g_num_sms;
     gather_rows_f16_kernel<<<(int)blocks, 256, 0, s>>>(p.a, p.sorted_token, p.T, p.K, p.S, p.a16,
                                                        p.err);
