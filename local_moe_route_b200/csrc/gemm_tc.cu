@@ -63,8 +63,18 @@ constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
 constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output feature)
 
-constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3, W_EPI = 11;
-constexpr int THREADS = 15 * 32;
+constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3;
+// Dequantising warpgroups take the stages round-robin: two for gate/up,
+// three for down, whose units are short (K = n) and leave the MMA warp
+// waiting on dequantisation more often (measured: down 0.73 -> 0.67 ms at the
+// large shape with three, gate/up slightly slower).  Registers bound the
+// count: three groups fit at 96 registers per thread.
+template <int OP>
+struct Roles {
+  static constexpr int NWG = OP == 0 ? 2 : 3;
+  static constexpr int W_EPI = W_DQ + 4 * NWG;
+  static constexpr int THREADS = (W_EPI + 4) * 32;
+};
 
 constexpr int RAW_OFF = 0;                                        // [RAW_ST][2][RAW_BYTES]
 constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;           // [B_ST][B_BYTES]
@@ -214,7 +224,7 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int OP, bool ILV>
-__global__ void __launch_bounds__(tc::THREADS, 1)
+__global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
                           const __grid_constant__ CUtensorMap map_q1,
                           const __grid_constant__ CUtensorMap map_b, const TcArgs args) {
@@ -363,9 +373,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       if (!stop && leader) mma_commit(acc_full);
       __syncwarp();
     }
-  } else if (warp < W_EPI) {
+  } else if (warp < Roles<OP>::W_EPI) {
     // -------------------------------------------------------------- dequantise
-    const int wg = (warp - W_DQ) >> 2;       // takes the stages g with g % 2 == wg
+    constexpr int NWG = Roles<OP>::NWG;
+    const int wg = (warp - W_DQ) >> 2;       // takes the stages g with g % NWG == wg
     const int q = warp & 3;                  // TMEM lane quadrant
     const int r = q * 32 + lane;             // weight row within the slot
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
@@ -408,8 +419,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     };
     uint4 blk_c[2], blk_n[2];
     int key_c = -1, key_n = -1;              // unit * 65536 + first group of the block
-    int iu = 0, kb = wg;                     // unit and K block of stage g (KB >= 2)
-    for (int g = wg; g < total_stages; g += 2) {
+    int iu = 0, kb = wg;                     // unit and K block of stage g
+    while (kb >= KB) {
+      kb -= KB;
+      ++iu;
+    }
+    for (int g = wg; g < total_stages; g += NWG) {
       const int grp0 = (kb * BK) >> g_shift;
       const int key = (iu << 16) | (grp0 & ~(SB - 1));
       if (key != key_c) {
@@ -453,8 +468,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         sc2[mm][0] = __byte_perm(w, 0, sel);
         sc2[mm][1] = G == 32 ? __byte_perm(w, 0, 0x3232u) : sc2[mm][0];
       }
-      kb += 2;
-      if (kb >= KB) {
+      kb += NWG;
+      while (kb >= KB) {
         kb -= KB;
         ++iu;
       }
@@ -506,7 +521,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     // out: thread t gathers 8 features of token t and stores 16 bytes, while
     // the next unit's MMAs already run.
     const int q = warp & 3;
-    const int et = threadIdx.x - W_EPI * 32;          // 0..127
+    const int et = threadIdx.x - Roles<OP>::W_EPI * 32;   // 0..127
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     for (int i = 0; i < my_units; ++i) {
       const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
@@ -650,7 +665,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < g_num_sms ? max_units : g_num_sms);
-  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
+  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::Roles<OP>::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
   return cudaGetLastError();
 }
 
