@@ -100,11 +100,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// Async-proxy fences and copies
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
+// TMA copies
 // 2-D TMA tile load global -> shared, completion counted on `bar` in bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, uint64_t* bar) {
@@ -117,20 +113,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// 16-byte cp.async (L2 only); src_bytes = 0 fills the destination with zeros.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-// The barrier receives one arrival when all earlier cp.async of this thread
-// have landed (the arrival counts toward the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-               : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -204,27 +186,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 
-// 32 lanes x 16 consecutive fp32 columns (thread i: lane base + i).
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-
-// Registers written by an asynchronous tcgen05.ld must not be read before
-// tcgen05.wait::ld; passing them through this empty asm right after the wait
-// keeps the compiler from moving their uses above it.
-template <int N>
-__device__ __forceinline__ void reg_fence(uint32_t* r) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -247,20 +208,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// 4-byte cp.async (through L1) into shared memory, tracked by commit groups.
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -298,16 +245,8 @@ __device__ __forceinline__ uint32_t idesc_f32acc(uint32_t M, uint32_t N, uint32_
 }
 constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
 
-// Offset of 16-byte chunk `c` (0..7) of row `r` in a K-major 128B-swizzled
-// tile whose rows are 128 bytes.
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
-  return ((r >> 3) << 10) | ((r & 7u) << 7) | (((c ^ (r & 7u)) & 7u) << 4);
-}
-
 // ---------------------------------------------------------------------------
 // Warp helpers
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-
 // True in exactly one lane of the (fully converged) warp.
 __device__ __forceinline__ bool elect_one() {
   uint32_t p;

@@ -63,7 +63,7 @@ constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
 constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output feature)
 
-constexpr int W_TMA = 0, W_MMA = 1, W_GATHER = 2, W_DQ = 3;
+constexpr int W_TMA = 0, W_MMA = 1, W_BTMA = 2, W_DQ = 3;
 // Dequantising warpgroups take the stages round-robin: two for gate/up,
 // three for down, whose units are short (K = n) and leave the MMA warp
 // waiting on dequantisation more often (measured: down 0.73 -> 0.67 ms at the
@@ -82,8 +82,7 @@ constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;                   // [2 * BM][ST
 constexpr int STG_BYTES = 2 * BM * STG_PITCH * 2;
 constexpr int BAR_OFF = STG_OFF + STG_BYTES;
 constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
-constexpr int TOK_OFF = BAR_OFF + NBARS * 8;
-constexpr int MISC_OFF = TOK_OFF + NT * 4;
+constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
 constexpr int SMEM = 1024 + MISC_OFF + 64;
 
 constexpr uint32_t TMEM_COLS = 512;
@@ -310,7 +309,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         }
       }
     }
-  } else if (warp == W_GATHER) {
+  } else if (warp == W_BTMA) {
     // -------------------------------------------------------------- token rows (B)
     // one TMA tile of 128 grouped rows per stage (rows past the unit belong
     // to other units or lie beyond S; the MMA reads only nrows of them)
