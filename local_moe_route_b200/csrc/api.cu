@@ -198,8 +198,13 @@ strata_status_t do_gemm(int op, const uint16_t* a, const int32_t* sorted_token,
   p.G = d.group;
   p.err = err;
   p.h_interleaved = h_interleaved;
-  const cudaError_t e = d.T <= kStreamMaxTokens ? launch_gemm_stream(p, sch, s)
-                                                : launch_gemm_tc(p, sch, s);
+  cudaError_t e;
+  if (d.T > kStreamMaxTokens) {
+    e = launch_gemm_tc(p, sch, s);
+  } else {
+    e = launch_gemm_decode(p, sch, s);
+    if (e == cudaErrorNotSupported) e = launch_gemm_stream(p, sch, s);
+  }
   return cuda_status(e);
 }
 

@@ -73,6 +73,9 @@ struct GemmProblem {
 };
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
+// Decode batches with K % 256 == 0 and N % 64 == 0 (weights staged by TMA);
+// cudaErrorNotSupported for other shapes.
+cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 
 // ---- combine
 cudaError_t launch_combine_checked(const uint16_t* rows, const float* w, const int32_t* slot_row,

@@ -351,16 +351,20 @@ def test_chunking_matches_whole_batch(dev):
     assert d <= GATE * y.float().pow(2).mean().sqrt().item()
 
 
-def test_deterministic(dev):
-    L = layer_for("default", dev)
+@pytest.mark.parametrize("name", ["default", "large", "verify4", "decode1"])
+def test_deterministic(name, dev):
+    # tensor-core path (default, large) and decode path with K split across
+    # warps and the split-summed small-batch router (verify4, decode1)
+    L = layer_for(name, dev)
     ws = sm.workspace(L.dims, dev)
     y1, i1, w1 = L.forward(ws=ws)
     y2, i2, w2 = L.forward(ws=ws)
     assert torch.equal(y1, y2) and torch.equal(i1, i2) and torch.equal(w1, w2)
 
 
-def test_cuda_graph_replay(dev):
-    L = layer_for("default", dev)
+@pytest.mark.parametrize("name", ["default", "verify4"])
+def test_cuda_graph_replay(name, dev):
+    L = layer_for(name, dev)
     ws = sm.workspace(L.dims, dev)
     y_eager, _, _ = L.forward(ws=ws)
     T, d = L.dims["T"], L.dims["d"]
