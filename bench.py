@@ -37,7 +37,7 @@ from moe_inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at T=6144, 512 experts top-10; % of tensor/HBM roofline"
 KERNEL_SOURCES = ["local_moe_route_b200/csrc/gemm_tc.cu", "local_moe_route_b200/csrc/common.cuh",
-                  "local_moe_route_b200/csrc/gemm_stream.cu"]
+                  "local_moe_route_b200/csrc/gemm_stream.cu", "local_moe_route_b200/csrc/gemm_decode.cu"]
 
 
 def log(*a):
@@ -364,7 +364,7 @@ def run_ours(args, wl):
         dur = stage_ms["gate_up"] / 1e3
         achieved = bytes_ / dur / 1e9
         roof = {"bound": "hbm",
-                "kernel": "gate/up step: work lists + moe_gemm_q4_stream_kernel<2> "
+                "kernel": "gate/up step: work lists + moe_gemm_q4_decode_kernel<2> "
                           "(gate/up + SwiGLU), one entry-point call",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_kind": f"{peak_kind} copy bandwidth",
