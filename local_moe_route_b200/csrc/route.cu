@@ -25,14 +25,14 @@ namespace rt {
 constexpr int BM = 128;                 // tokens per CTA (TMEM lanes)
 constexpr int BN = 128;                 // experts per CTA (TMEM columns)
 constexpr int BK = 64;                  // K per stage (one 128-byte swizzle row)
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;                // 99 KB of shared memory: two CTAs per SM
 constexpr int A_BYTES = BM * BK * 2;    // x tile       16 KB
 constexpr int B_BYTES = BN * BK * 2;    // W_r tile     16 KB (two 64-expert boxes)
 constexpr int SMEM = 1024 + STAGES * (A_BYTES + B_BYTES) + 256;
 constexpr int THREADS = 192;            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 }  // namespace rt
 
-__global__ void __launch_bounds__(rt::THREADS, 1)
+__global__ void __launch_bounds__(rt::THREADS, 2)
     router_logits_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                             const __grid_constant__ CUtensorMap map_wr, int T, int d, int E,
                             float* __restrict__ logits, unsigned* err) {
@@ -85,12 +85,19 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f32acc(BM, BN, kFmtBF16, 1);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(&full[s], (kb / STAGES) & 1, abort_flag, err)) break;
-        tc_fence_after();
+    // the whole warp follows the ring; one lane, elected once, issues the
+    // MMAs and commits
+    const bool leader = elect_one();
+    const uint32_t idesc = idesc_f32acc(BM, BN, kFmtBF16, 1);
+    bool stop = false;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait_warp(&full[s], (kb / STAGES) & 1, abort_flag, err)) {
+        stop = true;
+        break;
+      }
+      tc_fence_after();
+      if (leader) {
         const uint32_t a0 = smem_addr(sA + s * A_BYTES);
         const uint32_t b0 = smem_addr(sB + s * B_BYTES);
 #pragma unroll
@@ -101,8 +108,9 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
         }
         mma_commit(&empty[s]);
       }
-      mma_commit(accf);
+      __syncwarp();
     }
+    if (!stop && leader) mma_commit(accf);
     __syncwarp();
   } else {
     const int q = warp & 3;          // TMEM lane quadrant this warp may read
