@@ -36,8 +36,14 @@ sys.path.insert(0, ROOT)
 from moe_inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at T=6144, 512 experts top-10; % of tensor/HBM roofline"
-KERNEL_SOURCES = ["local_moe_route_b200/csrc/gemm_tc.cu", "local_moe_route_b200/csrc/common.cuh",
-                  "local_moe_route_b200/csrc/gemm_stream.cu", "local_moe_route_b200/csrc/gemm_decode.cu"]
+# Sources each profiled kernel is built from: its DRAM counters in
+# profiles/traffic.json stand only while these files are unchanged.
+KERNEL_SOURCES = {
+    "gemm_gate_up_large": ["local_moe_route_b200/csrc/gemm_tc.cu",
+                           "local_moe_route_b200/csrc/common.cuh"],
+    "gemm_gate_up_verify4": ["local_moe_route_b200/csrc/gemm_decode.cu",
+                             "local_moe_route_b200/csrc/common.cuh"],
+}
 
 
 def log(*a):
@@ -125,9 +131,9 @@ def launches_per_step(T, d, E):
     return n
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -151,7 +157,7 @@ def profiled_traffic(kernel):
     with open(path) as f:
         t = json.load(f)
     e = t.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -414,7 +420,7 @@ def run_ours(args, wl):
         dur = stage_ms["gate_up"] / 1e3
         achieved = bytes_ / dur / 1e9
         roof = {"bound": "hbm",
-                "kernel": "gate/up step: work lists + moe_gemm_q4_decode_kernel<2> "
+                "kernel": "gate/up step: work lists + moe_gemm_q4_decode_kernel<2, G> "
                           "(gate/up + SwiGLU), one entry-point call",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_kind": f"{peak_kind} copy bandwidth",

@@ -6,7 +6,7 @@
 // "两天移植，预填充提速8倍：Strata引擎实测", section "Strata快在哪", decode
 // paragraph), so the work is bound by HBM bandwidth over those bytes.  Here a
 // producer warp keeps a ring of shared-memory stages full with bulk tensor
-// copies -- the bytes in flight no longer depend on registers -- and four
+// copies -- the bytes in flight no longer depend on registers -- and eight
 // consumer warps turn each stage into mma.sync fragments:
 //   * a unit is 64 output features of one expert (gate and up both for
 //     gate/up); a stage holds, per weight matrix, 64 rows x 256 K (128 bytes
@@ -15,11 +15,13 @@
 //   * consumer warp w owns rows 16 (w % 4) .. + 15 and one half of each
 //     stage's K (w / 4); the two halves' fp32 sums meet in shared memory at
 //     the end of the unit and are added in a fixed order;
-//   * nibble pairs (i, i + 4) become exact integer fragments with one shift,
-//     one mask-and-or and one fma each; the K order inside each 32-wide
-//     half-block is permuted identically for the token operand; each MMA
-//     covers one 32-wide half-block, i.e. one scale group, and the fp16 group
-//     scale multiplies the fp32 partial sum.
+//   * nibble pairs (i, i + 4) become exact integer fragments with one
+//     mask-and-xor and one fma each (plus one shift per packed word for fp16,
+//     three for bf16); the K order inside each 32-wide half-block is
+//     permuted identically for the token operand;
+//   * the MMAs of one scale group (32, 64 or 128 K, a compile-time constant)
+//     sum integer codes times token values in fp32, and the group's fp16
+//     scale multiplies that sum once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -52,21 +54,40 @@ struct DecodeArgs {
   const uint16_t* s1;
   const float* row_scale;
   uint16_t* out;
-  int T, K, N, G;
+  int T, K, N;
   unsigned* err;
 };
 
+// The eight int4 codes of one packed word (K order 0..7, low nibble first)
+// as four exact integer pairs: pair i holds codes (i, i + 4), in the low and
+// high half of the register.  The mask-and-xor flips each code's sign bit
+// and sets the exponent in one logic op, giving 1024 + (q + 8) (fp16) or
+// 128 + (q + 8) (bf16), and one fma removes the offset.  fp16 takes codes 1
+// and 3 straight from bits 4..7 as 1024 + 16 (q + 8) -- exact, 16 (q + 8) <=
+// 240 fits the 10-bit mantissa -- and the same fma scales them back by 1/16,
+// which saves two shifts per word; bf16's 7-bit mantissa has no room for
+// that.
 template <bool F16>
-__device__ __forceinline__ uint32_t dk_pair(uint32_t wx, int i) {
-  uint32_t q;
+__device__ __forceinline__ void dk_word(uint32_t w, uint32_t (&p)[4]) {
   if (F16) {
-    const uint32_t v = ((wx >> (4 * i)) & 0x000F000Fu) | 0x64006400u;   // 1024 + (q + 8)
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
+    const uint32_t w8 = w >> 8;
+    const uint32_t v0 = (w & 0x000F000Fu) ^ 0x64086408u;
+    const uint32_t v1 = (w & 0x00F000F0u) ^ 0x64806480u;
+    const uint32_t v2 = (w8 & 0x000F000Fu) ^ 0x64086408u;
+    const uint32_t v3 = (w8 & 0x00F000F0u) ^ 0x64806480u;
+    // 1.0, -1032 and 1/16, -72 (fp16 pairs)
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[0]) : "r"(v0), "r"(0x3C003C00u), "r"(0xE408E408u));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[1]) : "r"(v1), "r"(0x2C002C00u), "r"(0xD480D480u));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[2]) : "r"(v2), "r"(0x3C003C00u), "r"(0xE408E408u));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[3]) : "r"(v3), "r"(0x2C002C00u), "r"(0xD480D480u));
   } else {
-    const uint32_t v = ((wx >> (4 * i)) & 0x000F000Fu) | 0x43004300u;   // 128 + (q + 8)
-    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x43084308u;
+      // 1.0, -136 (bf16 pairs)
+      asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p[i]) : "r"(v), "r"(0x3F803F80u), "r"(0xC308C308u));
+    }
   }
-  return q;
 }
 
 template <bool F16>
@@ -86,50 +107,28 @@ __device__ __forceinline__ void dk_mma(float (&c)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 32-wide half-block of one matrix: packed words of rows g and g + 8
-// (nibbles XORed with 8 inside), two MMAs, the group scales applied to the
-// fp32 partial sums.
-template <bool F16>
-__device__ __forceinline__ void dk_half(float (&acc)[4], uint32_t wg, uint32_t wg8, float sg,
-                                        float sg8, uint32_t b00, uint32_t b01, uint32_t b10,
-                                        uint32_t b11) {
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
-  wg ^= 0x88888888u;
-  wg8 ^= 0x88888888u;
-  dk_mma<F16>(c, dk_pair<F16>(wg, 0), dk_pair<F16>(wg8, 0), dk_pair<F16>(wg, 1),
-              dk_pair<F16>(wg8, 1), b00, b01);
-  dk_mma<F16>(c, dk_pair<F16>(wg, 2), dk_pair<F16>(wg8, 2), dk_pair<F16>(wg, 3),
-              dk_pair<F16>(wg8, 3), b10, b11);
-  acc[0] = fmaf(sg, c[0], acc[0]);
-  acc[1] = fmaf(sg, c[1], acc[1]);
-  acc[2] = fmaf(sg8, c[2], acc[2]);
-  acc[3] = fmaf(sg8, c[3], acc[3]);
-}
-
-// Group scales of one row for one stage (KC / G consecutive groups: 8, 4 or
-// 2 fp16 values), one aligned load.
-__device__ __forceinline__ uint4 dk_scales(const uint16_t* p, int groups) {
-  uint4 v = make_uint4(0, 0, 0, 0);
-  if (groups == 8) {
-    v = ld_nc_v4(p);
-  } else if (groups == 4) {
-    const uint2 t = ld_nc_v2(p);
-    v.x = t.x;
-    v.y = t.y;
-  } else {
+// Group scales of one row for one consumer warp's half of a stage (128 K:
+// 128 / G consecutive fp16 values), one aligned load.
+template <int G>
+__device__ __forceinline__ uint2 dk_scales(const uint16_t* p) {
+  uint2 v = make_uint2(0, 0);
+  if (G == 32)
+    v = ld_nc_v2(p);
+  else if (G == 64)
     v.x = ld_nc_u32(p);
-  }
+  else
+    v.x = ld_nc_u16(p);
   return v;
 }
 
-__device__ __forceinline__ float dk_scale_at(const uint4& v, int idx) {
-  const int w = idx >> 1;
-  const uint32_t x = (w & 2) ? ((w & 1) ? v.w : v.z) : ((w & 1) ? v.y : v.x);
-  return __half2float(__ushort_as_half(static_cast<unsigned short>((idx & 1) ? (x >> 16) : x)));
+// Scale j of those (j is a constant once the caller's loop is unrolled).
+__device__ __forceinline__ float dk_scale_at(const uint2& v, int j) {
+  const uint32_t x = (j & 2) ? v.y : v.x;
+  return __half2float(__ushort_as_half(static_cast<unsigned short>((j & 1) ? (x >> 16) : x)));
 }
 
-template <int NMAT>
-__global__ void __launch_bounds__(dk::THREADS)
+template <int NMAT, int G>
+__global__ void __launch_bounds__(dk::THREADS, NMAT == 1 ? 3 : 2)
     moe_gemm_q4_decode_kernel(const __grid_constant__ CUtensorMap map_w0,
                               const __grid_constant__ CUtensorMap map_w1,
                               const __grid_constant__ CUtensorMap map_x, const DecodeArgs args) {
@@ -143,7 +142,7 @@ __global__ void __launch_bounds__(dk::THREADS)
   uint64_t* empty = full + ST;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + ST);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = args.K, N = args.N, G = args.G;
+  const int K = args.K, N = args.N;
   const int NKC = K / KC;                    // stages per unit
   const int FBK = N / ROWS;                  // units per expert
   const int units = (*args.n_active) * FBK;
@@ -218,11 +217,12 @@ __global__ void __launch_bounds__(dk::THREADS)
     }
   } else {
     // ------------------------------------------------------------ consumers
+    constexpr int NG = 128 / G;              // scale groups in a warp's half of a stage
+    constexpr int HPG = G / 32;              // 32-K half-blocks per group
     const int g8 = lane >> 2, t = lane & 3;
     const int rg = warp & 3, kh = warp >> 2;   // row group, half of the stage's K
     const int r0 = rg * 16 + g8;             // rows r0 and r0 + 8 of the unit
     float* red = reinterpret_cast<float*>(smem + Lay::RED_OFF) + (rg * 32 + lane) * 8;
-    const int GS = KC / G;                   // scale groups per stage
     const int swz = (r0 & 7) << 4;           // 128-byte swizzle (row r0 + 8 alike)
     uint32_t gst = 0;
     bool failed = false;                     // uniform over the consumer warps
@@ -232,20 +232,23 @@ __global__ void __launch_bounds__(dk::THREADS)
       const int fb = u % FBK;
       const int p_begin = args.offsets[e];
       const int cnt_all = args.offsets[e + 1] - p_begin;
-      const size_t srow = (size_t)(e * N + fb * ROWS + r0) * (K / G);
+      // this warp's first scale of row r0: group (kc 256 + kh 128) / G of the row
+      const size_t srow = (size_t)(e * N + fb * ROWS + r0) * (K / G) + kh * NG;
       const size_t srow8 = srow + (size_t)8 * (K / G);
       for (int c0 = 0; c0 < cnt_all && !failed; c0 += XROWS) {
       const int cnt = min(XROWS, cnt_all - c0);
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-      uint4 sc[2][2];                        // [matrix][row r0 / r0 + 8], next stage
+      float acc[NMAT][4];
+      uint2 sc[NMAT][2];                     // [matrix][row r0 / r0 + 8], next stage
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
         const uint16_t* sp = m == 0 ? args.s0 : args.s1;
-        sc[m][0] = dk_scales(sp + srow, GS);
-        sc[m][1] = dk_scales(sp + srow8, GS);
+        sc[m][0] = dk_scales<G>(sp + srow);
+        sc[m][1] = dk_scales<G>(sp + srow8);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[m][q] = 0.f;
       }
       for (int kc = 0; kc < NKC; ++kc, ++gst) {
-        uint4 cur[2][2];
+        uint2 cur[NMAT][2];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
           cur[m][0] = sc[m][0];
@@ -255,35 +258,44 @@ __global__ void __launch_bounds__(dk::THREADS)
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             const uint16_t* sp = m == 0 ? args.s0 : args.s1;
-            sc[m][0] = dk_scales(sp + srow + (size_t)(kc + 1) * GS, GS);
-            sc[m][1] = dk_scales(sp + srow8 + (size_t)(kc + 1) * GS, GS);
+            sc[m][0] = dk_scales<G>(sp + srow + (size_t)(kc + 1) * (2 * NG));
+            sc[m][1] = dk_scales<G>(sp + srow8 + (size_t)(kc + 1) * (2 * NG));
           }
         }
         const int s = gst % ST;
         if (!mbar_wait_warp(&full[s], (gst / ST) & 1, abort_flag, args.err)) break;
         const uint8_t* st = smem + s * Lay::STAGE;
-        const uint8_t* xs = st + NMAT * WBYTES + g8 * (KC * 2);
+        const uint8_t* xs = st + NMAT * WBYTES + g8 * (KC * 2) + kh * 256;
+        float c[NMAT][4];                    // one scale group's integer-code sums
 #pragma unroll
-        for (int kk = 0; kk < KC / 128; ++kk) {
-          const int kb = kh * (KC / 128) + kk;   // this warp's 64-K blocks of the stage
+        for (int hb = 0; hb < 4; ++hb) {     // 32-K half-blocks of this warp's 128 K
+          const int chunk = kh * 4 + hb;     // 16-byte chunk of the 128-byte row
+          const uint4 x = *reinterpret_cast<const uint4*>(xs + (hb * 32 + t * 8) * 2);
+          // B fragments: K slots (2t, 2t+1) <- elements (i, i+4), (2t+8, 2t+9) <- (i+1, i+5)
+          const uint32_t b00 = __byte_perm(x.x, x.z, 0x5410);
+          const uint32_t b01 = __byte_perm(x.x, x.z, 0x7632);
+          const uint32_t b10 = __byte_perm(x.y, x.w, 0x5410);
+          const uint32_t b11 = __byte_perm(x.y, x.w, 0x7632);
+          const int off = ((chunk << 4) ^ swz) + t * 4;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int c = kb * 2 + h;        // 16-byte chunk of the 128-byte row
-            const uint4 x = *reinterpret_cast<const uint4*>(xs + (kb * 64 + h * 32 + t * 8) * 2);
-            // B fragments: K slots (2t, 2t+1) <- elements (i, i+4), (2t+8, 2t+9) <- (i+1, i+5)
-            const uint32_t b00 = __byte_perm(x.x, x.z, 0x5410);
-            const uint32_t b01 = __byte_perm(x.x, x.z, 0x7632);
-            const uint32_t b10 = __byte_perm(x.y, x.w, 0x5410);
-            const uint32_t b11 = __byte_perm(x.y, x.w, 0x7632);
-            const int gi = (kb * 64 + h * 32) / G;   // group within the stage
-            const int off = ((c << 4) ^ swz) + t * 4;
+          for (int m = 0; m < NMAT; ++m) {
+            const uint8_t* W = st + m * WBYTES;
+            uint32_t p0[4], p1[4];
+            dk_word<F16>(*reinterpret_cast<const uint32_t*>(W + r0 * 128 + off), p0);
+            dk_word<F16>(*reinterpret_cast<const uint32_t*>(W + (r0 + 8) * 128 + off), p1);
+            if (hb % HPG == 0) {
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-              const uint8_t* W = st + m * WBYTES;
-              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(W + r0 * 128 + off);
-              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(W + (r0 + 8) * 128 + off);
-              dk_half<F16>(m == 0 ? acc0 : acc1, w0, w1, dk_scale_at(cur[m][0], gi),
-                           dk_scale_at(cur[m][1], gi), b00, b01, b10, b11);
+              for (int q = 0; q < 4; ++q) c[m][q] = 0.f;
+            }
+            dk_mma<F16>(c[m], p0[0], p1[0], p0[1], p1[1], b00, b01);
+            dk_mma<F16>(c[m], p0[2], p1[2], p0[3], p1[3], b10, b11);
+            if (hb % HPG == HPG - 1) {       // group complete: apply its fp16 scales
+              const int j = hb / HPG;
+              const float s0 = dk_scale_at(cur[m][0], j), s8 = dk_scale_at(cur[m][1], j);
+              acc[m][0] = fmaf(s0, c[m][0], acc[m][0]);
+              acc[m][1] = fmaf(s0, c[m][1], acc[m][1]);
+              acc[m][2] = fmaf(s8, c[m][2], acc[m][2]);
+              acc[m][3] = fmaf(s8, c[m][3], acc[m][3]);
             }
           }
         }
@@ -298,8 +310,8 @@ __global__ void __launch_bounds__(dk::THREADS)
       if (kh == 1) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          red[q] = acc0[q];
-          red[4 + q] = acc1[q];
+          red[q] = acc[0][q];
+          if (NMAT == 2) red[4 + q] = acc[NMAT - 1][q];
         }
       }
       named_barrier_sync(1, CONSUMERS * 32);
@@ -307,8 +319,8 @@ __global__ void __launch_bounds__(dk::THREADS)
       if (kh == 0) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          acc0[q] += red[q];
-          acc1[q] += red[4 + q];
+          acc[0][q] += red[q];
+          if (NMAT == 2) acc[NMAT - 1][q] += red[4 + q];
         }
       }
       named_barrier_sync(1, CONSUMERS * 32);   // red is reused by the next tile
@@ -322,10 +334,10 @@ __global__ void __launch_bounds__(dk::THREADS)
         if (col < cnt) {
           float v;
           if (NMAT == 2) {
-            const float gv = acc0[q], uv = acc1[q];
+            const float gv = acc[0][q], uv = acc[NMAT - 1][q];
             v = gv / (1.0f + __expf(-gv)) * uv;
           } else {
-            v = acc0[q];
+            v = acc[0][q];
             if (args.row_scale) v *= args.row_scale[p_begin + c0 + col];
           }
           args.out[(size_t)(p_begin + c0 + col) * N + feat] = f16_bits(v);
@@ -336,12 +348,38 @@ __global__ void __launch_bounds__(dk::THREADS)
   }
 }
 
+// One CTA per unit up to as many as fit on the GPU at once (three per SM for
+// down, two for gate/up, by shared memory and registers).
+template <int NMAT, int G>
+static cudaError_t launch_decode(const CUtensorMap& mw0, const CUtensorMap& mw1,
+                                 const CUtensorMap& mx, const DecodeArgs& a, long units,
+                                 int num_sms, cudaStream_t s) {
+  using namespace dk;
+  auto kern = moe_gemm_q4_decode_kernel<NMAT, G>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<NMAT>::SMEM);
+  if (e != cudaSuccess) return e;
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, Layout<NMAT>::SMEM);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+  }
+  long blocks = units;
+  if (blocks > (long)per_sm * num_sms) blocks = (long)per_sm * num_sms;
+  if (blocks < 1) blocks = 1;
+  kern<<<(int)blocks, THREADS, Layout<NMAT>::SMEM, s>>>(mw0, mw1, mx, a);
+  return cudaSuccess;
+}
+
 // Takes the problem if its shapes fit the staged kernel (K a multiple of 256,
 // N of 64); otherwise returns cudaErrorNotSupported and the caller uses the
 // register-streaming kernel.
 cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
   using namespace dk;
-  if (p.K % KC != 0 || p.N % ROWS != 0 || p.T > XROWS) return cudaErrorNotSupported;
+  if (p.K % KC != 0 || p.N % ROWS != 0 || p.T > XROWS ||
+      (p.G != 32 && p.G != 64 && p.G != 128))
+    return cudaErrorNotSupported;
   static int num_sms = 0;
   if (num_sms == 0) {
     int dev = 0;
@@ -379,23 +417,20 @@ cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaSt
   a.T = p.T;
   a.K = p.K;
   a.N = p.N;
-  a.G = p.G;
   a.err = p.err;
   const int max_active = p.S < p.E ? p.S : p.E;
-  long blocks = (long)max_active * (p.N / ROWS);
-  if (blocks > 2L * num_sms) blocks = 2L * num_sms;
-  if (blocks < 1) blocks = 1;
+  const long units = (long)max_active * (p.N / ROWS);
+  cudaError_t e = cudaSuccess;
   if (gu) {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_decode_kernel<2>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<2>::SMEM);
-    if (e != cudaSuccess) return e;
-    moe_gemm_q4_decode_kernel<2><<<(int)blocks, THREADS, Layout<2>::SMEM, s>>>(mw0, mw1, mx, a);
+    if (p.G == 32) e = launch_decode<2, 32>(mw0, mw1, mx, a, units, num_sms, s);
+    else if (p.G == 64) e = launch_decode<2, 64>(mw0, mw1, mx, a, units, num_sms, s);
+    else e = launch_decode<2, 128>(mw0, mw1, mx, a, units, num_sms, s);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_decode_kernel<1>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<1>::SMEM);
-    if (e != cudaSuccess) return e;
-    moe_gemm_q4_decode_kernel<1><<<(int)blocks, THREADS, Layout<1>::SMEM, s>>>(mw0, mw1, mx, a);
+    if (p.G == 32) e = launch_decode<1, 32>(mw0, mw1, mx, a, units, num_sms, s);
+    else if (p.G == 64) e = launch_decode<1, 64>(mw0, mw1, mx, a, units, num_sms, s);
+    else e = launch_decode<1, 128>(mw0, mw1, mx, a, units, num_sms, s);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
