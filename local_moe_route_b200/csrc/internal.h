@@ -73,8 +73,8 @@ struct GemmProblem {
 };
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
-// Decode batches with K % 256 == 0 and N % 64 == 0 (weights staged by TMA);
-// cudaErrorNotSupported for other shapes.
+// Decode batches with K % 256 == 0, N % 64 == 0 and a group of 32, 64 or 128
+// (weights staged by TMA); cudaErrorNotSupported for other shapes.
 cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 
 // ---- combine
