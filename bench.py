@@ -85,9 +85,15 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        return self.summarise(self.lines)
+
+    @staticmethod
+    def summarise(lines):
+        """Median SM clock under load, the maximum clock and the throttle
+        reasons seen active, from nvidia-smi CSV lines in FIELDS order."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue

@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py (CPU only): the clock record that decides
+whether a timed run is kept, the committed DRAM-traffic records and the
+launch count it claims."""
+import json
+import os
+
+import pytest
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _line(sm, mx=1965, reasons=("Not Active",) * 4):
+    # index, clocks.sm, clocks.max.sm, power.draw, active mask, 4 reasons
+    return ", ".join(["0", str(sm), str(mx), "812.5", "0x0000000000000000", *reasons])
+
+
+def test_clock_summary_median_under_load_and_no_reasons():
+    lines = [_line(345), _line(1965), _line(1950), _line(1965), _line(1965)]
+    c = bench.ClockSampler.summarise(lines)
+    # the idle sample (below half of max) is left out of the median
+    assert c == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 5}
+
+
+def test_clock_summary_reports_each_active_reason():
+    act = ("Not Active", "Active", "Not Active", "Active")   # hw_thermal, sw_power_cap
+    lines = [_line(1500), _line(1490, reasons=act), "garbled", _line("[N/A]")]
+    c = bench.ClockSampler.summarise(lines)
+    assert c["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert c["samples"] == 2 and c["sm_mhz"] == pytest.approx(1495.0)
+
+
+def test_clock_summary_without_samples_is_none():
+    assert bench.ClockSampler.summarise([]) is None
+    assert bench.ClockSampler.summarise(["not, a, sample"]) is None
+
+
+def test_traffic_records_name_existing_sources():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    assert rec, "no traffic records"
+    for kernel, e in rec.items():
+        assert kernel in bench.KERNEL_SOURCES, kernel
+        for p in bench.KERNEL_SOURCES[kernel]:
+            assert os.path.exists(os.path.join(ROOT, p)), p
+        assert e["dram_bytes_per_launch"] > 0
+        assert len(e["source_hash"]) == 16
+
+
+def test_traffic_record_is_void_once_its_sources_change(monkeypatch, tmp_path):
+    assert bench.profiled_traffic("no_such_kernel") is None
+    kernel = "gemm_gate_up_large"
+    stored = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+    if stored["source_hash"] != bench.kernel_source_hash(kernel):
+        pytest.skip("record already void for the working tree's sources")
+    assert bench.profiled_traffic(kernel) == stored["dram_bytes_per_launch"]
+    extra = tmp_path / "changed.cu"
+    extra.write_text("// one more source\n")
+    monkeypatch.setitem(bench.KERNEL_SOURCES, kernel,
+                        bench.KERNEL_SOURCES[kernel] + [str(extra)])
+    assert bench.profiled_traffic(kernel) is None
+
+
+@pytest.mark.parametrize("T,d,E,want", [
+    (6144, 4096, 512, 10),   # tensor-core router, x copied to fp16 for the GEMM
+    (512, 4096, 128, 10),
+    (100, 4096, 128, 10),    # CUDA-core router without K split (T > 16)
+    (16, 4096, 512, 11),     # K-split router + split reduction, tensor-core GEMM
+    (8, 4096, 512, 10),      # K-split router, decode GEMM (no fp16 copy)
+    (1, 32, 8, 9),           # one K split: no reduction kernel
+])
+def test_launch_count_follows_dispatch_rules(T, d, E, want):
+    assert bench.launches_per_step(T, d, E) == want
