@@ -30,6 +30,22 @@ static unsigned* check_word_ptr() {
   return cache[dev];
 }
 
+// Streaming multiprocessors of the current device, looked up once per device.
+int sm_count() {
+  static std::mutex mu;
+  static int cache[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                         uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle,

@@ -22,6 +22,8 @@
 //   * the MMAs of one scale group (32, 64 or 128 K, a compile-time constant)
 //     sum integer codes times token values in fp32, and the group's fp16
 //     scale multiplies that sum once.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -359,11 +361,13 @@ static cudaError_t launch_decode(const CUtensorMap& mw0, const CUtensorMap& mw1,
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<NMAT>::SMEM);
   if (e != cudaSuccess) return e;
-  static int per_sm = 0;
+  static std::atomic<int> per_sm_cache{0};   // the same on every B200
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
   if (per_sm == 0) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, Layout<NMAT>::SMEM);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
   }
   long blocks = units;
   if (blocks > (long)per_sm * num_sms) blocks = (long)per_sm * num_sms;
@@ -380,13 +384,7 @@ cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaSt
   if (p.K % KC != 0 || p.N % ROWS != 0 || p.T > XROWS ||
       (p.G != 32 && p.G != 64 && p.G != 128))
     return cudaErrorNotSupported;
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (num_sms <= 0) num_sms = 148;
-  }
+  const int num_sms = sm_count();
   CUtensorMap mw0, mw1, mx;
   const uint64_t rows = (uint64_t)p.E * p.N;
   if (encode_tmap_2d(&mw0, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q0, p.K / 2, rows, p.K / 2, KC / 2, ROWS,

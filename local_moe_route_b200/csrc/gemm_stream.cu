@@ -250,13 +250,7 @@ __global__ void __launch_bounds__(st::THREADS, 2)
 }
 
 cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (num_sms <= 0) num_sms = 148;
-  }
+  const int num_sms = sm_count();
   StreamArgs a;
   a.a = p.a;
   a.a_rows = p.op == 0 ? p.T : p.S;

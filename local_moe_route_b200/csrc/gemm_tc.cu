@@ -604,8 +604,6 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   }
 }
 
-static int g_num_sms = 0;
-
 template <int OP, bool ILV>
 static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
   CUtensorMap m0, m1;
@@ -632,16 +630,11 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM);
     if (e != cudaSuccess) return e;
   }
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
+  const int num_sms = sm_count();
   if (OP == 0) {
     // the gate/up B operand: fp16 rows of x in grouped order
     long blocks = (p.S + 7) / 8;                     // 8 rows (warps) per block
-    if (blocks > 16L * g_num_sms) blocks = 16L * g_num_sms;
+    if (blocks > 16L * num_sms) blocks = 16L * num_sms;
     gather_rows_f16_kernel<<<(int)blocks, 256, 0, s>>>(p.a, p.sorted_token, p.T, p.K, p.S, p.a16,
                                                        p.err);
   }
@@ -663,7 +656,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   a.err = p.err;
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
-  const int grid = (int)(max_units < g_num_sms ? max_units : g_num_sms);
+  const int grid = (int)(max_units < num_sms ? max_units : num_sms);
   moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::Roles<OP>::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
   return cudaGetLastError();
 }

@@ -28,6 +28,9 @@ inline int max_tiles(int S, int E) {
   return S / kTileRows + (S < E ? S : E) + 1;
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count();
+
 // Resolves a driver entry point once (the tensor-map encoder).
 CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
