@@ -8,6 +8,7 @@ import torch
 
 import local_moe_route_b200 as sm
 from moe_inputs import chunk_sizes, make_custom, make_inputs
+from parity_metrics import gate_error, half_ulp, raw_error, rms, round_to, vs_rounded  # noqa: F401
 
 _WEIGHTS = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
 
@@ -146,31 +147,6 @@ class Layer:
 def assert_device_ok():
     torch.cuda.synchronize()
     assert sm.strata_moe_device_status() == sm.STRATA_OK
-
-
-def rms(a):
-    return float(np.sqrt(np.mean(np.square(a))))
-
-
-def half_ulp(ref: np.ndarray, fmt: str) -> np.ndarray:
-    """Half a unit in the last place of |ref| in the output format: the error a
-    correctly rounded result may carry on top of the computation's own."""
-    mant = {"bf16": 8, "fp16": 11}[fmt]
-    tiny = {"bf16": 2.0 ** -133, "fp16": 2.0 ** -25}[fmt]
-    e = np.floor(np.log2(np.maximum(np.abs(ref), 1e-300)))
-    return np.maximum(2.0 ** (e - mant), tiny)
-
-
-def gate_error(got: np.ndarray, ref: np.ndarray, fmt: str) -> float:
-    """max(|got - ref| - half_ulp(ref)) / RMS(ref); the gate is <= 1.5e-2.
-    A value that is exact but for its final rounding scores <= 0."""
-    excess = np.abs(got - ref) - half_ulp(ref, fmt)
-    return float(np.max(excess) / max(rms(ref), 1e-30))
-
-
-def raw_error(got: np.ndarray, ref: np.ndarray) -> float:
-    """max |got - ref| / RMS(ref), reported alongside the gate."""
-    return float(np.max(np.abs(got - ref)) / max(rms(ref), 1e-30))
 
 
 def near_tie_tokens(logits: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:
