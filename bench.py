@@ -3,7 +3,7 @@
 with SwiGLU -> combine) through the library's C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference]
+                    [--impl ours|reference] [--sustain-s S] [--no-secondary]
 
 One step = one strata_moe_forward over one batch of the workload (default:
 the 6144-token prefill chunk, d=4096, 512 experts, top-10, n=1024, int4 with
@@ -13,6 +13,16 @@ JSON line.  With N > 1 (torchrun), every rank runs an independent replica
 (the layer shards by token batches with no exchange); the time is the max over
 ranks and `value` the total tokens of all ranks per second.
 
+At N = 1 the line also carries
+  * `secondary`: the other workloads of the same model family, each timed on
+    its own inputs -- the 4-token verify batch and the 1-token decode step
+    (HBM roofline over the weights they touch), the 512-token default batch
+    (both rooflines) and the whole 34,000-token skewed prompt as six chunks
+    (tokens/s = 34,000 / sum of chunk times, per-chunk expert load);
+  * `sustained`: the headline forward run back to back for --sustain-s
+    seconds (default 60) with nvidia-smi sampled every 200 ms: the rate, the
+    median SM clock, time x clock, and step times binned by clock.
+
 --impl reference times the fp64 CPU oracle on a bounded token sample of the
 same workload on the host cores (rank 0 only).
 """
@@ -20,7 +30,6 @@ same workload on the host cores (rank 0 only).
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -33,7 +42,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import WORKLOADS, make_inputs  # noqa: E402
+from moe_inputs import WORKLOADS, Workload, chunk_sizes, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at T=6144, 512 experts top-10; % of tensor/HBM roofline"
 # Sources each profiled kernel is built from: its DRAM counters in
@@ -44,6 +53,7 @@ KERNEL_SOURCES = {
     "gemm_gate_up_verify4": ["local_moe_route_b200/csrc/gemm_decode.cu",
                              "local_moe_route_b200/csrc/common.cuh"],
 }
+WEIGHTS = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
 
 
 def log(*a):
@@ -52,15 +62,17 @@ def log(*a):
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi every 200 ms while the timed region runs."""
+    """Samples nvidia-smi every 200 ms while a timed region runs; every line
+    is kept with the host time it arrived."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host time, csv line)
 
     def start(self):
         try:
@@ -75,7 +87,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def stop(self):
         if self.proc is None:
@@ -85,26 +97,37 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        return self.summarise(self.lines)
+        return self.summarise([ln for _, ln in self.lines])
 
-    @staticmethod
-    def summarise(lines):
+    @classmethod
+    def parse(cls, line):
+        """(sm MHz, max MHz, power W, set of active reasons) or None."""
+        f = [x.strip() for x in line.split(",")]
+        if len(f) < 9:
+            return None
+        try:
+            sm, mx = float(f[1]), float(f[2])
+        except ValueError:
+            return None
+        try:
+            pw = float(f[3])
+        except ValueError:
+            pw = None
+        reasons = {nm for nm, v in zip(cls.REASONS, f[5:9]) if v.lower() == "active"}
+        return sm, mx, pw, reasons
+
+    @classmethod
+    def summarise(cls, lines):
         """Median SM clock under load, the maximum clock and the throttle
         reasons seen active, from nvidia-smi CSV lines in FIELDS order."""
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in lines:
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            p = cls.parse(line)
+            if p is None:
                 continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
+            sm.append(p[0])
+            mx = p[1]
+            reasons |= p[3]
         if not sm:
             return None
         busy = [v for v in sm if mx and v > 0.5 * mx] or sm
@@ -118,7 +141,7 @@ def device_layer(inp, dev):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     L = {"x": t(inp["x"]).view(torch.bfloat16), "w_router": t(inp["w_router"]).view(torch.bfloat16),
          "bias": None if inp.get("bias") is None else t(inp["bias"])}
-    for n in ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s"):
+    for n in WEIGHTS:
         L[n] = t(inp[n])
     return L
 
@@ -135,6 +158,22 @@ def launches_per_step(T, d, E):
     n += 1                   # down
     n += 1                   # combine
     return n
+
+
+def expert_bytes(wl):
+    """Packed int4 codes and fp16 group scales of one expert's three matrices."""
+    return 3 * wl.n * wl.d // 2 + 3 * wl.n * (wl.d // wl.group) * 2
+
+
+def layer_flops(wl, T):
+    """Algorithmic FLOPs of the layer for T tokens: the k chosen experts'
+    three projections plus the router."""
+    return 2.0 * T * wl.k * 3 * wl.d * wl.n + 2.0 * T * wl.d * wl.E
+
+
+def layer_hbm_bytes(wl, T, touched):
+    """Algorithmic bytes: weights of the touched experts, W_r, x and y."""
+    return touched * expert_bytes(wl) + wl.d * wl.E * 2 + 2 * T * wl.d * 2
 
 
 def kernel_source_hash(kernel):
@@ -186,6 +225,88 @@ def job_throughput(tokens_per_rank, world, max_ms):
     return tokens_per_rank * world / (max_ms / 1e3)
 
 
+# --------------------------------------------------------------------------- timing
+class LayerRun:
+    """One workload resident on the device, called through strata_moe_forward.
+    Batches of at most 64 tokens replay the forward as one CUDA graph (ten
+    short kernels would otherwise wait on host launch overhead) and, since
+    the weights they touch can stay in L2 from one step to the next, are
+    timed one step at a time after a 256 MB write that evicts L2."""
+
+    def __init__(self, sm, wl, inp, dev, T=None):
+        import torch
+        self.sm, self.wl, self.dev = sm, wl, dev
+        self.T = wl.T if T is None else T
+        self.L = device_layer(inp, dev)
+        self.dims = wl.dims(self.T)
+        self.ws = sm.workspace(self.dims, dev)
+        self.y = torch.empty((self.T, wl.d), dtype=torch.bfloat16, device=dev)
+        self.q4 = [(self.L[n + "_q"], self.L[n + "_s"]) for n in ("gate", "up", "down")]
+        self.graph = None
+        self.flush = None
+        if self.T <= 64:
+            self.forward()
+            torch.cuda.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph):
+                self.forward()
+            torch.cuda.synchronize()
+            self.flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+
+    def forward(self, x=None, out=None, T=None, ids=None):
+        import torch
+        dims = self.dims if T is None else self.wl.dims(T)
+        st = self.sm.strata_moe_forward(self.L["x"] if x is None else x, self.L["w_router"],
+                                        self.L["bias"], *self.q4, dims,
+                                        self.y if out is None else out, ids, None, self.ws,
+                                        stream=torch.cuda.current_stream())
+        if st != self.sm.STRATA_OK:
+            raise self.sm.StrataError(st, "forward")
+
+    def step(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.forward()
+
+    def time(self, steps):
+        """Per-step device times (ms), CUDA events on the launching stream."""
+        import torch
+        stream = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        for i in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            ev[2 * i].record(stream)
+            self.step()
+            ev[2 * i + 1].record(stream)
+        torch.cuda.synchronize()
+        return [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
+
+    def touched(self):
+        """Experts the batch routes to (from one forward's ids)."""
+        import torch
+        ids = torch.empty((self.T, self.wl.k), dtype=torch.int32, device=self.dev)
+        self.forward(ids=ids)
+        torch.cuda.synchronize()
+        return ids.cpu().numpy()
+
+
+def expert_load(ids, E):
+    counts = np.bincount(ids.ravel(), minlength=E)
+    used = counts[counts > 0]
+    return {"experts_touched": int(used.size), "rows_max": int(used.max()),
+            "rows_mean_touched": round(float(used.mean()), 2),
+            "rows_mean_all": round(float(counts.mean()), 2)}
+
+
+def roof(achieved, peak, unit, bound, kind, **extra):
+    out = {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+           "frac": round(achieved / peak, 4), "peak_kind": kind}
+    out.update(extra)
+    return out
+
+
 # --------------------------------------------------------------------------- our arm
 def run_ours(args, wl):
     import torch
@@ -204,36 +325,13 @@ def run_ours(args, wl):
     sm.lib()                                       # fails loudly without the library
 
     inp = make_inputs(wl)
-    L = device_layer(inp, dev)
-    dims = wl.dims()
+    R = LayerRun(sm, wl, inp, dev)
+    L, dims, ws, y = R.L, R.dims, R.ws, R.y
     T, d, k, n, E = wl.T, wl.d, wl.k, wl.n, wl.E
     S = T * k
-    ws = sm.workspace(dims, dev)
-    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-    gate, up, down = (L["gate_q"], L["gate_s"]), (L["up_q"], L["up_s"]), (L["down_q"], L["down_s"])
+    gate, up, down = R.q4
     stream = torch.cuda.current_stream()
-
-    def forward(x=None, out=None):
-        st = sm.strata_moe_forward(L["x"] if x is None else x, L["w_router"], L["bias"], gate, up,
-                                   down, dims, y if out is None else out, None, None, ws,
-                                   stream=torch.cuda.current_stream())
-        if st != sm.STRATA_OK:
-            raise sm.StrataError(st, "forward")
-
-    # Small batches (decode / verify) replay the forward as one CUDA graph:
-    # ten short kernels would otherwise wait on host launch overhead.  Large
-    # batches launch eagerly (the GPU is the bottleneck there).
-    graph = None
-    if T <= 64:
-        forward()
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            forward()
-        torch.cuda.synchronize()
-    step = graph.replay if graph is not None else forward
-    # weights a small batch touches can fit in L2; those runs flush it
-    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if T <= 64 else None
+    forward = R.forward
 
     def barrier():
         torch.cuda.synchronize()
@@ -243,19 +341,19 @@ def run_ours(args, wl):
 
     # ---- headline: K forwards, device time
     for _ in range(args.warmup):
-        step()
+        R.step()
     clocks = ClockSampler(dev.index) if rank == 0 else None
     barrier()
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    if flush is None:
+    if R.flush is None:
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
         ev0.record(stream)
         step_ev[0].record(stream)
         for i in range(args.steps):
-            step()
+            R.step()
             step_ev[i + 1].record(stream)
         ev1.record(stream)
         barrier()
@@ -264,15 +362,8 @@ def run_ours(args, wl):
     else:
         # the touched weights would stay in L2 from one step to the next:
         # overwrite L2 between steps and time each step alone
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
-        for a_, b_ in pairs:
-            flush.zero_()
-            a_.record(stream)
-            step()
-            b_.record(stream)
+        step_ms = R.time(args.steps)
         barrier()
-        step_ms = [a_.elapsed_time(b_) for a_, b_ in pairs]
         total_ms = max_over_ranks(sum(step_ms), dev)
     clk = clocks.stop() if clocks else None
     assert sm.strata_moe_device_status(stream) == sm.STRATA_OK
@@ -320,80 +411,15 @@ def run_ours(args, wl):
     per = {nm: [] for nm in names}
     for _ in range(args.steps):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        if R.flush is not None:
+            R.flush.zero_()
         staged(evs)
         torch.cuda.synchronize()
         for i, nm in enumerate(names):
             per[nm].append(evs[i].elapsed_time(evs[i + 1]))
     stage_ms = {nm: statistics.mean(v) for nm, v in per.items()}
 
-    # ---- end to end: host x -> device, forward, y -> host, every step
-    x_host = torch.from_numpy(inp["x"]).view(torch.bfloat16).pin_memory()
-    if flush is not None:
-        # small batches: one step at a time, L2 flushed before each, each
-        # step (copy in, forward, copy out) timed alone
-        y_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-        x_dev = torch.empty_like(L["x"])
-        for _ in range(args.warmup):
-            x_dev.copy_(x_host, non_blocking=True)
-            forward(x_dev)
-            y_host.copy_(y, non_blocking=True)
-        barrier()
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
-        for a_, b_ in pairs:
-            flush.zero_()
-            a_.record(stream)
-            x_dev.copy_(x_host, non_blocking=True)
-            forward(x_dev)
-            y_host.copy_(y, non_blocking=True)
-            b_.record(stream)
-        barrier()
-        e2e_elapsed = sum(a_.elapsed_time(b_) for a_, b_ in pairs)
-    else:
-        # large batches: copies pipelined against compute.  Step i's input is
-        # copied in on one stream and its output copied out on another while
-        # the forward of the neighbouring step runs; two device buffers each.
-        y_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-        x_dev = [torch.empty_like(L["x"]) for _ in range(2)]
-        y_dev = [torch.empty_like(y) for _ in range(2)]
-        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
-        ev = lambda: torch.cuda.Event()
-        x_free = [ev(), ev()]      # forward that read x_dev[b] is done
-        y_free = [ev(), ev()]      # copy-out of y_dev[b] is done
-        for b_ in range(2):
-            x_free[b_].record(stream)
-            y_free[b_].record(stream)
-
-        def e2e_step(i):
-            b_ = i & 1
-            x_in, fwd_done = ev(), ev()
-            with torch.cuda.stream(h2d):
-                h2d.wait_event(x_free[b_])
-                x_dev[b_].copy_(x_host, non_blocking=True)
-                x_in.record(h2d)
-            stream.wait_event(x_in)
-            stream.wait_event(y_free[b_])
-            forward(x_dev[b_], out=y_dev[b_])
-            fwd_done.record(stream)
-            x_free[b_].record(stream)
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(fwd_done)
-                y_host[b_].copy_(y_dev[b_], non_blocking=True)
-                y_free[b_].record(d2h)
-
-        for i in range(args.warmup):
-            e2e_step(i)
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            e2e_step(i)
-        stream.wait_event(y_free[0])
-        stream.wait_event(y_free[1])
-        e1.record(stream)
-        barrier()
-        e2e_elapsed = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_elapsed, dev)
+    e2e_ms = max_over_ranks(time_e2e(R, inp, args, stream, barrier), dev)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -404,45 +430,26 @@ def run_ours(args, wl):
     tokens = T * args.steps * world
     value = job_throughput(T * args.steps, world, total_ms)
     ms_step = total_ms / args.steps
-    tensor_bound = T > 8
-    if tensor_bound:
+    ids_np = R.touched()
+    touched = int(np.unique(ids_np).size)
+    if T > 8:
         # dominant kernel: gate/up grouped GEMM; algorithmic FLOPs per launch
         flops = 2.0 * S * 2 * d * n
-        dur = stage_ms["gate_up"] / 1e3
-        achieved = flops / dur / 1e12
-        roof = {"bound": "tensor",
-                "kernel": "gate/up step: work lists + grouped fp16 copy of x + "
-                          "moe_gemm_q4_tc_kernel<0,0> (gate/up + SwiGLU), one entry-point call",
-                "achieved": round(achieved, 1), "peak": tf_burst, "unit": "TFLOP/s",
-                "frac": round(achieved / tf_burst, 4),
-                "peak_kind": f"{peak_kind} bf16 dense burst (fp16 dense is the same rate)",
-                "algorithmic_per_launch": flops,
-                "traffic": profiled_traffic("gemm_gate_up_" + wl.name)}
+        roofline = roof(flops / (stage_ms["gate_up"] / 1e3) / 1e12, tf_burst, "TFLOP/s", "tensor",
+                        f"{peak_kind} bf16 dense burst (fp16 dense is the same rate)",
+                        kernel="gate/up step: " + gate_up_kernels(T),
+                        algorithmic_per_launch=flops,
+                        traffic=profiled_traffic("gemm_gate_up_" + wl.name))
     else:
-        ids_np = ids.cpu().numpy()
-        touched = len(np.unique(ids_np))
-        per_expert = (2 * n * d // 2 + 2 * n * (d // wl.group) * 2 + d * n // 2 + d * (n // wl.group) * 2)
-        bytes_ = touched * per_expert * 2 / 3        # gate+up share of the touched experts
-        dur = stage_ms["gate_up"] / 1e3
-        achieved = bytes_ / dur / 1e9
-        roof = {"bound": "hbm",
-                "kernel": "gate/up step: work lists + moe_gemm_q4_decode_kernel<2, G> "
-                          "(gate/up + SwiGLU), one entry-point call",
-                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "peak_kind": f"{peak_kind} copy bandwidth",
-                "algorithmic_per_launch": bytes_,
-                "traffic": profiled_traffic("gemm_gate_up_" + wl.name)}
-    layer_flops = 2.0 * S * 3 * d * n + 2.0 * T * d * E
-    layer_roof = None
-    if not tensor_bound:
-        # the whole layer against HBM: weights of the experts the batch touches,
-        # the router matrix, x and y, over the step time
-        per_exp = 3 * n * d // 2 + 3 * n * (d // wl.group) * 2
-        lbytes = touched * per_exp + d * E * 2 + 2 * T * d * 2
-        lach = lbytes / (ms_step / 1e3) / 1e9
-        layer_roof = {"bound": "hbm", "achieved": round(lach, 1), "peak": hbm, "unit": "GB/s",
-                      "frac": round(lach / hbm, 4), "bytes_per_step": lbytes,
-                      "experts_touched": touched}
+        # gate+up share of the touched experts' weight bytes
+        bytes_ = touched * expert_bytes(wl) * 2 / 3
+        roofline = roof(bytes_ / (stage_ms["gate_up"] / 1e3) / 1e9, hbm, "GB/s", "hbm",
+                        f"{peak_kind} copy bandwidth",
+                        kernel="gate/up step: " + gate_up_kernels(T),
+                        algorithmic_per_launch=bytes_,
+                        traffic=profiled_traffic("gemm_gate_up_" + wl.name))
+    lflops = layer_flops(wl, T)
+    lbytes = layer_hbm_bytes(wl, T, touched)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -451,39 +458,306 @@ def run_ours(args, wl):
         "config": {"workload": wl.name, "T": T, "d": d, "E": E, "k": k, "n": n,
                    "group": wl.group, "router_bias": wl.zipf > 0,
                    "l2": ("L2 flushed between steps (256 MB write), each step timed alone"
-                          if flush is not None else
+                          if R.flush is not None else
                           "inputs larger than L2 (3.4 GB of weights), no flush"),
-                   "launch": "one CUDA graph per forward" if graph is not None else "eager",
+                   "launch": "one CUDA graph per forward" if R.graph is not None else "eager",
                    "parallelism": f"replicas x{world}"},
-        "layer_tflops": round(layer_flops / (ms_step / 1e3) / 1e12, 1),
+        "layer_tflops": round(lflops / (ms_step / 1e3) / 1e12, 1),
         "step_ms": {"min": round(min(step_ms), 4), "median": round(statistics.median(step_ms), 4),
                     "max": round(max(step_ms), 4)},
         "stage_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
-        "roofline": roof,
-        "layer_roofline": layer_roof,
+        "roofline": roofline,
+        "layer_roofline": {
+            "tensor": roof(lflops / (ms_step / 1e3) / 1e12, tf_burst, "TFLOP/s", "tensor",
+                           f"{peak_kind} bf16 dense burst", flops_per_step=lflops),
+            "hbm": roof(lbytes / (ms_step / 1e3) / 1e9, hbm, "GB/s", "hbm",
+                        f"{peak_kind} copy bandwidth", bytes_per_step=lbytes,
+                        experts_touched=touched)},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
         "gpu_launches": launches_per_step(T, d, E) * args.steps,
         "clocks": clk,
     }
+    if world == 1 and not args.no_secondary:
+        out["secondary"] = {}
+        for name in ("verify4", "decode1", "default", "skewed"):
+            if name != wl.name:
+                out["secondary"][name] = run_secondary(sm, dev, WORKLOADS[name], args)
+    if world == 1 and args.sustain_s > 0:
+        out["sustained"] = run_sustained(R, args.sustain_s, dev, tf_burst, tf_sus, peak_kind)
     if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_tokens)
+        R.forward()
+        out["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_tokens, R.y)
     return out
 
 
+def gate_up_kernels(T):
+    if T > 8:
+        return ("work lists + grouped fp16 copy of x + moe_gemm_q4_tc_kernel<0,0> "
+                "(gate/up + SwiGLU), one entry-point call")
+    return "work lists + moe_gemm_q4_decode_kernel<2, G> (gate/up + SwiGLU), one entry-point call"
+
+
+def time_e2e(R, inp, args, stream, barrier):
+    """Same forward with the host -> device copy of x (pinned memory) and the
+    device -> host copy of y inside the timed region, every step."""
+    import torch
+    T, d = R.T, R.wl.d
+    x_host = torch.from_numpy(inp["x"]).view(torch.bfloat16).pin_memory()
+    if R.flush is not None:
+        # small batches: one step at a time, L2 flushed before each, each
+        # step (copy in, forward, copy out) timed alone
+        y_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(R.L["x"])
+        for _ in range(args.warmup):
+            x_dev.copy_(x_host, non_blocking=True)
+            R.forward(x_dev)
+            y_host.copy_(R.y, non_blocking=True)
+        barrier()
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a_, b_ in pairs:
+            R.flush.zero_()
+            a_.record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            R.forward(x_dev)
+            y_host.copy_(R.y, non_blocking=True)
+            b_.record(stream)
+        barrier()
+        return sum(a_.elapsed_time(b_) for a_, b_ in pairs)
+    # large batches: copies pipelined against compute.  Step i's input is
+    # copied in on one stream and its output copied out on another while
+    # the forward of the neighbouring step runs; two device buffers each.
+    y_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(R.L["x"]) for _ in range(2)]
+    y_dev = [torch.empty_like(R.y) for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    x_free = [ev(), ev()]      # forward that read x_dev[b] is done
+    y_free = [ev(), ev()]      # copy-out of y_dev[b] is done
+    for b_ in range(2):
+        x_free[b_].record(stream)
+        y_free[b_].record(stream)
+
+    def e2e_step(i):
+        b_ = i & 1
+        x_in, fwd_done = ev(), ev()
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(x_free[b_])
+            x_dev[b_].copy_(x_host, non_blocking=True)
+            x_in.record(h2d)
+        stream.wait_event(x_in)
+        stream.wait_event(y_free[b_])
+        R.forward(x_dev[b_], out=y_dev[b_])
+        fwd_done.record(stream)
+        x_free[b_].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(fwd_done)
+            y_host[b_].copy_(y_dev[b_], non_blocking=True)
+            y_free[b_].record(d2h)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_event(y_free[0])
+    stream.wait_event(y_free[1])
+    e1.record(stream)
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+# --------------------------------------------------------------------------- secondary
+def run_secondary(sm, dev, wl, args):
+    """One other workload on its own seeded inputs: tokens/s and the layer's
+    rooflines.  The skewed prompt runs as its chunks, one forward each."""
+    import gc
+    import torch
+    hbm, tf_burst, _, peak_kind = measured_peaks()
+    inp = make_inputs(wl)
+    sizes = chunk_sizes(wl.T, wl.chunk)
+    R = LayerRun(sm, wl, inp, dev, T=max(sizes))
+    res = {"T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "n": wl.n, "group": wl.group}
+    steps = args.secondary_steps
+    if len(sizes) == 1:
+        for _ in range(args.warmup):
+            R.step()
+        ms = R.time(steps)
+        med = statistics.median(ms)
+        ids = R.touched()
+        load = expert_load(ids, wl.E)
+        lflops = layer_flops(wl, wl.T)
+        lbytes = layer_hbm_bytes(wl, wl.T, load["experts_touched"])
+        res.update({
+            "tokens_per_s": round(wl.T / (med / 1e3), 1), "ms_per_step": round(med, 4),
+            "steps": steps,
+            "step_ms": {"min": round(min(ms), 4), "max": round(max(ms), 4)},
+            "launch": "one CUDA graph per forward" if R.graph is not None else "eager",
+            "l2": "flushed (256 MB write) before each step" if R.flush is not None else
+                  "weights larger than L2, no flush",
+            "layer_roofline": {
+                "hbm": roof(lbytes / (med / 1e3) / 1e9, hbm, "GB/s", "hbm",
+                            f"{peak_kind} copy bandwidth", bytes_per_step=lbytes),
+                "tensor": roof(lflops / (med / 1e3) / 1e12, tf_burst, "TFLOP/s", "tensor",
+                               f"{peak_kind} bf16 dense burst", flops_per_step=lflops)},
+            "expert_load": load,
+        })
+    else:
+        # the whole prompt, chunk by chunk; per repetition the chunk times add
+        starts = np.concatenate([[0], np.cumsum(sizes)[:-1]]).astype(int)
+        xs = [R.L["x"][s0:s0 + m] for s0, m in zip(starts, sizes)]
+        ys = [torch.empty((m, wl.d), dtype=torch.bfloat16, device=dev) for m in sizes]
+        stream = torch.cuda.current_stream()
+
+        def prompt(evs=None):
+            for c, m in enumerate(sizes):
+                if evs is not None:
+                    evs[c].record(stream)
+                R.forward(xs[c], out=ys[c], T=m)
+            if evs is not None:
+                evs[len(sizes)].record(stream)
+
+        for _ in range(max(1, args.warmup // 2)):
+            prompt()
+        reps = max(3, steps // 10)
+        per_chunk = [[] for _ in sizes]
+        totals = []
+        for _ in range(reps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(sizes) + 1)]
+            prompt(evs)
+            torch.cuda.synchronize()
+            t = [evs[c].elapsed_time(evs[c + 1]) for c in range(len(sizes))]
+            for c in range(len(sizes)):
+                per_chunk[c].append(t[c])
+            totals.append(sum(t))
+        med = statistics.median(totals)
+        chunks = []
+        for c, m in enumerate(sizes):
+            ids = torch.empty((m, wl.k), dtype=torch.int32, device=dev)
+            R.forward(xs[c], out=ys[c], T=m, ids=ids)
+            torch.cuda.synchronize()
+            load = expert_load(ids.cpu().numpy(), wl.E)
+            load.update({"T": m, "ms": round(statistics.median(per_chunk[c]), 4)})
+            chunks.append(load)
+        lflops = layer_flops(wl, wl.T)
+        res.update({
+            "tokens_per_s": round(wl.T / (med / 1e3), 1),
+            "ms_per_prompt": round(med, 4), "repetitions": reps,
+            "chunks": chunks, "launch": "eager, one forward per chunk",
+            "layer_roofline": {
+                "tensor": roof(lflops / (med / 1e3) / 1e12, tf_burst, "TFLOP/s", "tensor",
+                               f"{peak_kind} bf16 dense burst", flops_per_prompt=lflops)},
+        })
+    assert sm.strata_moe_device_status() == sm.STRATA_OK
+    del R
+    gc.collect()
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------------------- sustained
+def run_sustained(R, seconds, dev, tf_burst, tf_sus, peak_kind):
+    """The headline forward back to back for `seconds`, nvidia-smi sampled
+    every 200 ms.  Events every `block` steps give the step time over the run;
+    each clock sample is paired with the block running when it was taken."""
+    import torch
+    stream = torch.cuda.current_stream()
+    block = 20 if R.T > 64 else 200
+    clocks = ClockSampler(dev.index)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    evs = []
+    while time.time() - t_host0 < seconds:
+        for _ in range(block):
+            R.step()
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        evs.append(e)
+        if len(evs) > 4:
+            evs[-4].synchronize()      # keep the host at most a few blocks ahead
+    torch.cuda.synchronize()
+    clocks.stop()
+    ends = [ev0.elapsed_time(e) for e in evs]            # ms since start, per block
+    nsteps = block * len(evs)
+    total = ends[-1]
+    starts = [0.0] + ends[:-1]
+    block_ms = [(b - a) / block for a, b in zip(starts, ends)]
+    samples = []
+    for ts, line in clocks.lines:
+        p = ClockSampler.parse(line)
+        t = (ts - t_host0) * 1e3
+        if p is None or t < 0 or t > total:
+            continue
+        i = int(np.searchsorted(ends, t))
+        samples.append((p[0], block_ms[min(i, len(block_ms) - 1)], p[2], p[3]))
+    summ = ClockSampler.summarise([ln for _, ln in clocks.lines]) or {}
+    bins = {}
+    for mhz, ms, _, _ in samples:
+        key = int(mhz // 100 * 100)
+        bins.setdefault(key, []).append(ms)
+    flops = layer_flops(R.wl, R.T)
+    ms_step = total / nsteps
+    med_mhz = summ.get("sm_mhz")
+    watts = [s[2] for s in samples if s[2] is not None]
+    return {
+        "seconds": round(total / 1e3, 1), "steps": nsteps, "ms_per_step": round(ms_step, 4),
+        "tokens_per_s": round(R.T * nsteps / (total / 1e3), 1),
+        "layer_tflops": round(flops / (ms_step / 1e3) / 1e12, 1),
+        "frac_of_burst": round(flops / (ms_step / 1e3) / 1e12 / tf_burst, 4),
+        "frac_of_sustained": (round(flops / (ms_step / 1e3) / 1e12 / tf_sus, 4)
+                              if tf_sus else None),
+        "peak_kind": peak_kind,
+        "first_10pct_ms_per_step": round(statistics.mean(block_ms[:max(1, len(block_ms) // 10)]), 4),
+        "last_10pct_ms_per_step": round(statistics.mean(block_ms[-max(1, len(block_ms) // 10):]), 4),
+        "clocks": summ,
+        "ms_per_step_x_median_mhz": round(ms_step * med_mhz, 1) if med_mhz else None,
+        "power_w_median": round(statistics.median(watts), 1) if watts else None,
+        "by_clock_mhz": {str(k_): {"samples": len(v), "ms_per_step": round(statistics.mean(v), 4)}
+                         for k_, v in sorted(bins.items())},
+    }
+
+
 # --------------------------------------------------------------------------- oracle
-def cpu_baseline(wl, inp, ntok):
+def cpu_baseline(wl, inp, ntok, y_dev=None):
+    """The fp64 oracle on a seeded token sample, on all host cores.  With the
+    GPU's output y_dev of the same batch, the sample also gives the parity
+    of those tokens: the gate (error beyond one bf16 rounding), the literal
+    max-abs error and the distance from the correctly rounded oracle."""
     import oracle
     ntok = min(ntok, wl.T)
-    toks = np.random.default_rng(99).choice(wl.T, ntok, replace=False)
+    toks = np.sort(np.random.default_rng(99).choice(wl.T, ntok, replace=False))
     oracle.lib()
     t0 = time.perf_counter()
-    oracle.moe_forward(inp, wl.k, wl.group, tokens=toks)
+    ref = oracle.moe_forward(inp, wl.k, wl.group, tokens=toks)
     dt = time.perf_counter() - t0
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": round(ntok / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{ntok} of {wl.T} tokens (seeded); the oracle's cost per token does "
-                      f"not depend on T", "seconds": round(dt, 2)}
+    out = {"value": round(ntok / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{ntok} of {wl.T} tokens (seeded); the oracle's cost per token does "
+                     f"not depend on T", "seconds": round(dt, 2)}
+    if y_dev is not None:
+        import torch
+        bits = y_dev.view(torch.int16).cpu().numpy().view(np.uint16)[toks]
+        got = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        y = ref["y"]
+        r = float(np.sqrt(np.mean(y * y)))
+        m, e = np.frexp(y)
+        rounded = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)      # RNE to bf16
+        half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(y), 1e-300))) - 8)
+        out["parity_of_sample"] = {
+            "gate": round(float(np.max(np.abs(got - y) - half_ulp) / r), 5),
+            "raw_max_abs": round(float(np.max(np.abs(got - y)) / r), 5),
+            "exactly_rounded_raw_max_abs": round(float(np.max(np.abs(rounded - y)) / r), 5),
+            "vs_rounded_oracle_max_abs": round(float(np.max(np.abs(got - rounded)) / r), 5),
+            "limit": 1.5e-2, "unit": "RMS of the oracle output"}
+    return out
 
 
 def run_reference(args, wl):
@@ -530,6 +804,11 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=256)
     ap.add_argument("--ref-tokens", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads (N = 1 only)")
+    ap.add_argument("--secondary-steps", type=int, default=50)
+    ap.add_argument("--sustain-s", type=float, default=60.0,
+                    help="seconds of back-to-back forwards after the timed steps (N = 1; 0: off)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (profiling cases; not a bench line)")
     ap.add_argument("--experts", type=int, default=0,
@@ -541,12 +820,13 @@ def main():
         args.warmup = 3
     wl = WORKLOADS[args.workload]
     if args.tokens or args.experts:
-        from moe_inputs import Workload
         wl = Workload(**{**wl.__dict__, "T": args.tokens or wl.T, "E": args.experts or wl.E,
                          "name": f"{wl.name}_T{args.tokens or wl.T}_E{args.experts or wl.E}"})
+        args.no_secondary = True
+        args.sustain_s = 0
     if wl.chunk and wl.T > wl.chunk:
-        # a chunked workload is timed one chunk (the largest) at a time
-        from moe_inputs import Workload
+        # a chunked workload's headline is one chunk (the largest); the whole
+        # prompt is timed among the secondary results
         wl = Workload(**{**wl.__dict__, "T": wl.chunk, "name": wl.name + "_chunk"})
     res = run_reference(args, wl) if args.impl == "reference" else run_ours(args, wl)
     if res is not None:

@@ -72,3 +72,27 @@ def test_traffic_record_is_void_once_its_sources_change(monkeypatch, tmp_path):
 ])
 def test_launch_count_follows_dispatch_rules(T, d, E, want):
     assert bench.launches_per_step(T, d, E) == want
+
+
+def test_algorithmic_work_matches_the_workload_table():
+    from moe_inputs import WORKLOADS
+    large = WORKLOADS["large"]
+    # packed int4 of gate, up, down (3 * 4096 * 1024 / 2) + fp16 scales per group of 64
+    assert bench.expert_bytes(large) == 6_684_672
+    assert bench.layer_flops(large, 6144) == pytest.approx(1.572e12, rel=1e-3)
+    # 40 experts, the router matrix, x and y of four tokens
+    assert bench.layer_hbm_bytes(large, 4, 40) == 40 * 6_684_672 + 4096 * 512 * 2 + 2 * 4 * 4096 * 2
+
+
+def test_expert_load_counts_rows_per_expert():
+    import numpy as np
+    ids = np.array([[0, 3], [3, 5], [3, 0]])
+    assert bench.expert_load(ids, 8) == {"experts_touched": 3, "rows_max": 3,
+                                         "rows_mean_touched": 2.0, "rows_mean_all": 0.75}
+
+
+def test_clock_line_parse_keeps_power_and_reasons():
+    act = ("Not Active", "Not Active", "Not Active", "Active")
+    sm, mx, pw, reasons = bench.ClockSampler.parse(_line(1800, reasons=act))
+    assert (sm, mx, pw, reasons) == (1800.0, 1965.0, 812.5, {"sw_power_cap"})
+    assert bench.ClockSampler.parse("garbled") is None
