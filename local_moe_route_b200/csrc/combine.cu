@@ -75,4 +75,37 @@ cudaError_t launch_combine_checked(const uint16_t* rows, const float* w, const i
   return cudaGetLastError();
 }
 
+// dst[i] = src[index[i]] for rows of `width` 16-bit values (width % 8 == 0):
+// one warp per row, 16-byte loads and stores.  Indices outside [0, src_rows)
+// are reported (kErrIndex) and read row 0.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint16_t* __restrict__ src, const int32_t* __restrict__ index,
+                       int src_rows, int rows, int width, uint16_t* __restrict__ dst,
+                       unsigned* err) {
+  const int lane = threadIdx.x & 31;
+  const int cpr = width / 8;
+  bool bad = false;
+  for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < rows; i += gridDim.x * 8) {
+    int r = index[i];
+    if ((unsigned)r >= (unsigned)src_rows) {
+      bad = true;
+      r = 0;
+    }
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + (size_t)r * width);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)i * width);
+    for (int c = lane; c < cpr; c += 32) d4[c] = __ldg(s4 + c);
+  }
+  if (bad) atomicOr(err, kErrIndex);
+}
+
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* index, int src_rows,
+                               int rows, int width, uint16_t* dst, unsigned* err,
+                               cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  long blocks = (rows + 7) / 8;
+  if (blocks > 16L * sm_count()) blocks = 16L * sm_count();
+  gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(src, index, src_rows, rows, width, dst, err);
+  return cudaGetLastError();
+}
+
 }  // namespace strata
