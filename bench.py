@@ -146,18 +146,31 @@ def device_layer(inp, dev):
     return L
 
 
-def launches_per_step(T, d, E):
+def fused_decode(T, d, E, k, n, group):
+    """Whether strata_moe_forward runs the batch as one persistent launch
+    (mirrors the library's rule for batches of at most four tokens)."""
+    if not (1 <= T <= 4 and k <= 32 and E <= 1024 and group in (32, 64, 128)
+            and d % 1024 == 0 and n % 256 == 0):
+        return False
+    xbytes = (T * (d + 8) * 2 + 1023) // 1024 * 1024
+    smem = 3 * 16384 + xbytes + 8 * 32 * 8 * 4 + 128 + (2 * 128 + 4 * 1024 + 1 + 2 * 128 + 64) * 4
+    return smem + 1024 <= 113 * 1024
+
+
+def launches_per_step(T, d, E, k=10, n=1024, group=64):
     """Kernel launches of one strata_moe_forward (mirrors the dispatch rules)."""
-    n = 2                    # router logits + top-k/softmax
+    if fused_decode(T, d, E, k, n, group):
+        return 1             # the whole layer in one kernel (plus a 16-byte memset)
+    c = 2                    # router logits + top-k/softmax
     tc_router = T >= 128 and E % 128 == 0
     if not tc_router and T <= 16 and d // 32 > 1:
-        n += 1               # sum of the K-split partial logits
-    n += 3                   # permutation: histogram, scan, scatter
-    n += 1                   # expert work lists
-    n += 2 if T > 8 else 1   # gate/up (+ fp16 copy of x on the tensor-core path)
-    n += 1                   # down
-    n += 1                   # combine
-    return n
+        c += 1               # sum of the K-split partial logits
+    c += 3                   # permutation: histogram, scan, scatter
+    c += 1                   # expert work lists
+    c += 2 if T > 8 else 1   # gate/up (+ fp16 copy of x on the tensor-core path)
+    c += 1                   # down
+    c += 1                   # combine
+    return c
 
 
 def expert_bytes(wl):
@@ -432,7 +445,15 @@ def run_ours(args, wl):
     ms_step = total_ms / args.steps
     ids_np = R.touched()
     touched = int(np.unique(ids_np).size)
-    if T > 8:
+    lflops = layer_flops(wl, T)
+    lbytes = layer_hbm_bytes(wl, T, touched)
+    if fused_decode(T, d, E, k, n, wl.group):
+        # the forward is one kernel: its roofline is the layer's, over HBM
+        roofline = roof(lbytes / (ms_step / 1e3) / 1e9, hbm, "GB/s", "hbm",
+                        f"{peak_kind} copy bandwidth",
+                        kernel="moe_decode_fused_kernel<G> (the whole layer, one launch)",
+                        algorithmic_per_launch=lbytes, traffic=None)
+    elif T > 8:
         # dominant kernel: gate/up grouped GEMM; algorithmic FLOPs per launch
         flops = 2.0 * S * 2 * d * n
         roofline = roof(flops / (stage_ms["gate_up"] / 1e3) / 1e12, tf_burst, "TFLOP/s", "tensor",
@@ -448,8 +469,6 @@ def run_ours(args, wl):
                         kernel="gate/up step: " + gate_up_kernels(T),
                         algorithmic_per_launch=bytes_,
                         traffic=profiled_traffic("gemm_gate_up_" + wl.name))
-    lflops = layer_flops(wl, T)
-    lbytes = layer_hbm_bytes(wl, T, touched)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -475,7 +494,7 @@ def run_ours(args, wl):
                         experts_touched=touched)},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
-        "gpu_launches": launches_per_step(T, d, E) * args.steps,
+        "gpu_launches": launches_per_step(T, d, E, k, n, wl.group) * args.steps,
         "clocks": clk,
     }
     if world == 1 and not args.no_secondary:

@@ -249,11 +249,44 @@ STRATA_API strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t*
                                    void* ws, size_t ws_bytes,
                                    strata_stream_t stream);
 
+/* Row gather for the expert-parallel exchange (no counterpart on the pages):
+ *   dst[i] = src[index[i]],  i < rows, rows of `width` 16-bit values (bf16 or
+ *   fp16 bit patterns; width a multiple of 8)
+ *   src [src_rows][width], index [rows] int32, dst [rows][width]
+ * An index outside [0, src_rows) is reported through
+ * strata_moe_device_status() and reads row 0. */
+STRATA_API strata_status_t strata_moe_gather_rows(const uint16_t* src, const int32_t* index,
+                                       int32_t src_rows, int32_t rows, int32_t width,
+                                       uint16_t* dst, strata_stream_t stream);
+
 /* Synchronises `stream`, then reports (and clears) the device-side check word
  * of the current device: STRATA_OK, or STRATA_ERR_DEVICE_CHECK when a kernel
  * since the last call recorded an out-of-range index or a bounded wait that
  * timed out.  This is the one entry point that blocks the host. */
 STRATA_API strata_status_t strata_moe_device_status(strata_stream_t stream);
+
+/* Diagnostic: drives the library's bounded waits into their time limit on
+ * purpose and lets them give up, so that callers (and the tests) can see the
+ * failure path work on their device.  The pages have no counterpart; every
+ * wait in the kernels above is bounded in the same way (about one second),
+ * after which the kernel records a time-out in the device check word,
+ * releases what it holds and returns instead of spinning forever.
+ *   out      device int32[8] (16-byte aligned), written by the kernels:
+ *            out[0..3]  1 if wait w completed, 0 if it gave up (an mbarrier
+ *                       that nothing arrives on; warp 0 waits alone, warps
+ *                       1..3 wait as whole warps and see warp 0's abort;
+ *                       warp 1 holds 32 columns of tensor memory meanwhile)
+ *            out[4]     nanoseconds warp 0 waited before giving up
+ *            out[5]     1 once warp 1 released its tensor memory
+ *            out[6]     1 if a two-CTA grid barrier that one CTA never
+ *                       reaches completed, 0 if it gave up
+ *            out[7]     nanoseconds that barrier waited
+ *   sync_ws  device scratch of 16 bytes (16-byte aligned), overwritten
+ * Both kernels take about one second each.  Afterwards
+ * strata_moe_device_status() reports STRATA_ERR_DEVICE_CHECK (and clears it);
+ * the device stays usable. */
+STRATA_API strata_status_t strata_moe_selftest_wait(int32_t* out, void* sync_ws,
+                                         strata_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -22,7 +22,8 @@ __all__ = [
     "strata_moe_workspace_bytes", "strata_status_string", "strata_moe_route",
     "strata_moe_permute", "strata_moe_permute_static", "STRATA_PERMUTE_STATIC_SCRATCH_INTS",
     "strata_moe_expert_gemm_q4", "strata_moe_combine",
-    "strata_moe_forward", "strata_moe_device_status", "workspace",
+    "strata_moe_forward", "strata_moe_device_status", "strata_moe_selftest_wait",
+    "strata_moe_gather_rows", "workspace",
 ]
 
 STRATA_OK = 0
@@ -107,6 +108,11 @@ def lib() -> ctypes.CDLL:
     L.strata_moe_forward.restype = st
     L.strata_moe_device_status.argtypes = [vp]
     L.strata_moe_device_status.restype = st
+    L.strata_moe_selftest_wait.argtypes = [vp, vp, vp]
+    L.strata_moe_selftest_wait.restype = st
+    i32 = ctypes.c_int32
+    L.strata_moe_gather_rows.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    L.strata_moe_gather_rows.restype = st
     _lib = L
     return L
 
@@ -196,6 +202,15 @@ def strata_moe_forward(x, w_router, bias, gate, up, down, dims, y, topk_ids_out=
 
 def strata_moe_device_status(stream=None) -> int:
     return lib().strata_moe_device_status(_stream(stream))
+
+
+def strata_moe_selftest_wait(out, sync_ws, stream=None) -> int:
+    return lib().strata_moe_selftest_wait(_ptr(out), _ptr(sync_ws), _stream(stream))
+
+
+def strata_moe_gather_rows(src, index, src_rows, rows, width, dst, stream=None) -> int:
+    return lib().strata_moe_gather_rows(_ptr(src), _ptr(index), int(src_rows), int(rows),
+                                        int(width), _ptr(dst), _stream(stream))
 
 
 def workspace(dims, device="cuda"):

@@ -16,7 +16,12 @@ namespace strata {
 // Device-side check word (one per device that loads the library).
 __device__ unsigned g_check_word;
 
-static unsigned* check_word_ptr() {
+unsigned* check_word();
+static unsigned* check_word_ptr() { return check_word(); }
+
+// Device address of g_check_word on the current device, looked up once per
+// device and cached.
+unsigned* check_word() {
   static std::mutex mu;
   static unsigned* cache[128] = {};
   int dev = 0;
@@ -135,10 +140,10 @@ Schedule schedule_at(uint8_t* ws, const SchedRegions& r) {
   s.n_active = reinterpret_cast<int32_t*>(ws + r.n_active.off);
   return s;
 }
-// fp16 rows of x in grouped order [T*k][d], the B operand of the tensor-core
-// gate/up path (batches above the streaming threshold).
+// x in fp16, token order [T][d]: the tensor-core gate/up path (batches above
+// the streaming threshold) gathers its B rows from it.
 size_t x16_bytes(const strata_moe_dims_t& d) {
-  return d.T > kStreamMaxTokens ? (size_t)d.T * d.k * d.d * 2 : 0;
+  return d.T > kStreamMaxTokens ? (size_t)d.T * d.d * 2 : 0;
 }
 size_t gemm_scratch(const strata_moe_dims_t& d) {
   Layout L;
@@ -148,7 +153,7 @@ size_t gemm_scratch(const strata_moe_dims_t& d) {
 }
 
 struct ForwardLayout {
-  Region ids, w, partial, counts, offsets, sorted_token, slot_row, hist, x16, h, rows;
+  Region ids, w, partial, counts, offsets, sorted_token, slot_row, hist, x16, h, rows, fused;
   SchedRegions sched;
   size_t total;
 };
@@ -168,6 +173,9 @@ ForwardLayout forward_layout(const strata_moe_dims_t& d) {
   f.x16 = L.add(x16_bytes(d));
   f.h = L.add(S * (size_t)d.n * 2);
   f.rows = L.add(S * (size_t)d.d * 2);
+  f.fused = L.add(decode_fused_fits(d.T, d.d, d.E, d.k, d.n, d.group)
+                      ? decode_fused_scratch(d.T, d.d, d.E, d.k, d.n)
+                      : 0);
   f.total = L.total;
   return f;
 }
@@ -409,6 +417,13 @@ strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router, 
   uint16_t* rows = reinterpret_cast<uint16_t*>(at(f.rows));
   const Schedule sch = schedule_at(base, f.sched);
 
+  if (decode_fused_fits(dims.T, dims.d, dims.E, dims.k, dims.n, dims.group)) {
+    // a decode / verify batch: the whole layer in one persistent launch
+    const cudaError_t e = launch_decode_fused(
+        x, w_router, bias, gate.q, gate.s, up.q, up.s, down.q, down.s, dims.T, dims.d, dims.E,
+        dims.k, dims.n, dims.group, y, topk_ids_out, topk_w_out, at(f.fused), err, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
   st = do_route(x, w_router, bias, dims, ids, w, nullptr, reinterpret_cast<float*>(at(f.partial)),
                 err, s);
   if (st != STRATA_OK) return st;
@@ -426,6 +441,18 @@ strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router, 
   st = do_gemm(1, h, nullptr, offsets, down, none, nullptr, dims, rows, sch, x16, err, s, true);
   if (st != STRATA_OK) return st;
   return cuda_status(launch_combine_checked(rows, w, slot_row, dims.T, dims.k, dims.d, y, err, s));
+}
+
+strata_status_t strata_moe_gather_rows(const uint16_t* src, const int32_t* index,
+                                       int32_t src_rows, int32_t rows, int32_t width,
+                                       uint16_t* dst, strata_stream_t stream) {
+  if (src_rows < 0 || rows < 0 || width <= 0 || width % 8) return STRATA_ERR_INVALID_ARG;
+  if (rows == 0) return STRATA_OK;
+  if (src_rows == 0 || !ok_ptr(src) || !ok_ptr(index) || !ok_ptr(dst)) return STRATA_ERR_INVALID_ARG;
+  unsigned* err = check_word_ptr();
+  if (!err) return STRATA_ERR_CUDA;
+  return cuda_status(launch_gather_rows(src, index, src_rows, rows, width, dst, err,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 strata_status_t strata_moe_device_status(strata_stream_t stream) {

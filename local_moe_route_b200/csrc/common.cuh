@@ -57,15 +57,34 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// A thread whose phase has not completed sleeps in try_wait until it does, or
+// for at most this long: waiting warps then take no issue slots from the
+// warps that do the work (without a hint the hardware's own limit is short
+// enough that a wait becomes a busy loop).
+#ifndef STRATA_WAIT_HINT_NS
+#define STRATA_WAIT_HINT_NS 20000
+#endif
+constexpr uint32_t kWaitHintNs = STRATA_WAIT_HINT_NS;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if (kWaitHintNs > 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kWaitHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
@@ -99,6 +118,32 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// Grid-wide barrier for kernels whose CTAs are all resident (cooperative
+// launch).  Called by thread 0 of each CTA after a CTA-wide
+// barrier; sync[0] counts arrivals over the launch, barrier number b
+// completes at (b + 1) * gridDim.x.  Gives up (false) after kWaitLimitNs or
+// when another CTA has raised sync[2]; a time-out records kErrTimeout and
+// raises sync[2] so every CTA winds down.
+__device__ __forceinline__ bool grid_barrier_wait(unsigned* sync, int b, unsigned* err) {
+  __threadfence();
+  atomicAdd(&sync[0], 1u);
+  const unsigned target = (unsigned)(b + 1) * gridDim.x;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
+    unsigned v, ab;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(sync) : "memory");
+    if (v >= target) return true;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(sync + 2) : "memory");
+    if (ab) return false;
+    if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) break;
+    __nanosleep(100);
+  }
+  atomicOr(err, kErrTimeout);
+  atomicExch(&sync[2], 1u);
+  return false;
+}
+
+
 // ---------------------------------------------------------------------------
 // TMA copies
 // 2-D TMA tile load global -> shared, completion counted on `bar` in bytes.
@@ -109,6 +154,35 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (from l2_policy_*) for the bytes read.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int32_t x,
+                                                 int32_t y, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// Four rows of a 2-D tensor (the map's box is one row high) into four
+// consecutive box-sized rows of shared memory: columns x.. of rows r[0..3].
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int32_t x,
+                                            const int (&r)[4], uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+      "r"(smem_addr(bar))
+      : "memory");
+}
+
+// L2 policies: data read once (streamed weights) leaves L2 first.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -310,6 +384,11 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
 __device__ __forceinline__ uint16_t f16_bits(float v) {
   return __half_as_ushort(__float2half_rn(v));
 }
+
+// True when v does not survive the conversion to fp16: NaN, or a magnitude of
+// 65520 or more (the smallest that rounds to infinity; 65504 is the largest
+// finite fp16).
+__device__ __forceinline__ bool f16_overflows(float v) { return !(fabsf(v) < 65520.f); }
 
 // Two floats -> fp16 pair (each rounded to nearest even), lo in the low half.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(dk::THREADS, NMAT == 1 ? 3 : 2)
             v = acc[0][q];
             if (args.row_scale) v *= args.row_scale[p_begin + c0 + col];
           }
+          if (f16_overflows(v)) atomicOr(args.err, kErrRange);
           args.out[(size_t)(p_begin + c0 + col) * N + feat] = f16_bits(v);
         }
       }

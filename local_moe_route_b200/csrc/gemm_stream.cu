@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(st::THREADS, 2)
               v = acc0[i];
               if (args.row_scale) v *= args.row_scale[p_begin + col];
             }
+            if (f16_overflows(v)) atomicOr(args.err, kErrRange);
             args.out[(size_t)(p_begin + col) * N + feat] = f16_bits(v);
           }
         }

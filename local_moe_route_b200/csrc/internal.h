@@ -64,7 +64,7 @@ struct GemmProblem {
   const uint8_t* q0; const uint16_t* s0;  // gate (or down)
   const uint8_t* q1; const uint16_t* s1;  // up (gate/up only)
   const float* row_scale;       // down only, nullable
-  uint16_t* a16;                // scratch [T*k][d]: fp16 x rows in grouped order (TC gate/up)
+  uint16_t* a16;                // scratch [T][d]: x in fp16, token order (TC gate/up)
   uint16_t* out;
   int T, S, E, K, N, G;         // K reduction dim, N output features
   // Tensor-core path only, set by the fused forward: h travels between the
@@ -80,9 +80,23 @@ cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaSt
 // (weights staged by TMA); cudaErrorNotSupported for other shapes.
 cudaError_t launch_gemm_decode(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 
+// ---- the whole layer for batches of at most four tokens, one launch
+bool decode_fused_fits(int T, int d, int E, int k, int n, int G);
+size_t decode_fused_scratch(int T, int d, int E, int k, int n);
+cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                                const uint8_t* q_gate, const uint16_t* s_gate,
+                                const uint8_t* q_up, const uint16_t* s_up,
+                                const uint8_t* q_down, const uint16_t* s_down, int T, int d,
+                                int E, int k, int n, int G, uint16_t* y, int32_t* ids_out,
+                                float* w_out, void* scratch, unsigned* err, cudaStream_t s);
+
 // ---- combine
 cudaError_t launch_combine_checked(const uint16_t* rows, const float* w, const int32_t* slot_row,
                                    int T, int k, int d, uint16_t* y, unsigned* err,
                                    cudaStream_t s);
+
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* index, int src_rows,
+                               int rows, int width, uint16_t* dst, unsigned* err,
+                               cudaStream_t s);
 
 }  // namespace strata

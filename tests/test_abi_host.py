@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
         "strata_moe_workspace_bytes", "strata_status_string", "strata_moe_route",
         "strata_moe_permute", "strata_moe_permute_static", "strata_moe_expert_gemm_q4",
         "strata_moe_combine",
-        "strata_moe_forward", "strata_moe_device_status"}
+        "strata_moe_forward", "strata_moe_device_status", "strata_moe_selftest_wait",
+        "strata_moe_gather_rows"}
 
 
 def test_library_exports_every_declared_symbol():
@@ -59,8 +60,8 @@ LARGE = dict(T=6144, d=4096, E=512, k=10, n=1024, group=64)
 def test_workspace_bytes():
     n = sm.strata_moe_workspace_bytes(LARGE)
     S = 6144 * 10
-    # at least the per-row fp16 buffers: grouped x [S][d], h [S][n], rows [S][d]
-    rows = S * 4096 * 2 + S * 1024 * 2 + S * 4096 * 2
+    # at least the fp16 buffers: x in token order [T][d], h [S][n], rows [S][d]
+    rows = 6144 * 4096 * 2 + S * 1024 * 2 + S * 4096 * 2
     assert n >= rows
     assert n < rows + 64 * 2 ** 20
     assert n % 256 == 0

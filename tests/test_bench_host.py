@@ -69,6 +69,9 @@ def test_traffic_record_is_void_once_its_sources_change(monkeypatch, tmp_path):
     (16, 4096, 512, 11),     # K-split router + split reduction, tensor-core GEMM
     (8, 4096, 512, 10),      # K-split router, decode GEMM (no fp16 copy)
     (1, 32, 8, 9),           # one K split: no reduction kernel
+    (4, 4096, 512, 1),       # verify batch: the whole layer in one launch
+    (1, 4096, 512, 1),
+    (5, 4096, 512, 10),      # five tokens: separate kernels again
 ])
 def test_launch_count_follows_dispatch_rules(T, d, E, want):
     assert bench.launches_per_step(T, d, E) == want

@@ -342,6 +342,62 @@ def test_out_of_fp16_range_input_is_reported(dev):
     assert sm.strata_moe_device_status() == sm.STRATA_OK
 
 
+def _fill(L, name, value):
+    """Replace one weight tensor by a constant (codes as a byte, scales as fp16)."""
+    a = L.inp[name]
+    if name.endswith("_q"):
+        arr = np.full(a.shape, value, np.uint8)
+    else:
+        arr = np.full(a.shape, value, np.float16).view(np.uint16)
+    L.inp[name] = arr
+    L.w[name] = torch.from_numpy(arr).to(L.device)
+
+
+def _expect_range_report():
+    torch.cuda.synchronize()
+    assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
+    assert sm.strata_moe_device_status() == sm.STRATA_OK        # cleared
+
+
+@pytest.mark.parametrize("T", [40, 4])
+def test_fp16_overflow_of_h_is_reported(T, dev):
+    """x inside the fp16 range, but gate and up sums of 2560 make h = SiLU(g) * u
+    about 6.5e6, beyond fp16: the gate/up epilogue reports it (tensor-core path
+    at T = 40, decode path at T = 4)."""
+    L = Layer.custom(dev, T=T, d=256, E=8, k=2, n=128, group=64, seed=55)
+    for nm in ("gate", "up"):
+        _fill(L, nm + "_q", 0x11)                         # every code q = 1
+        _fill(L, nm + "_s", 0.01)
+    L.forward(torch.full_like(L.x, 1000.0))
+    _expect_range_report()
+
+
+@pytest.mark.parametrize("T", [40, 4])
+def test_fp16_overflow_of_down_rows_is_reported(T, dev):
+    """Finite fp16 h rows of 60000 against codes of 7 and scales of 0.02 give
+    per-row outputs near 1.1e6: the down epilogue reports them."""
+    L = Layer.custom(dev, T=T, d=256, E=8, k=2, n=128, group=64, seed=56)
+    _fill(L, "down_q", 0x77)
+    _fill(L, "down_s", 0.02)
+    S = T * 2
+    ids = np.stack([np.arange(T) % 8, (np.arange(T) + 1) % 8], axis=1).astype(np.int32)
+    _, offsets, _, _ = oracle.permute(ids, 8)
+    h = torch.full((S, 128), 60000.0, dtype=torch.float16, device=dev)
+    L.down(h, torch.from_numpy(offsets).to(dev), T)
+    _expect_range_report()
+
+
+def test_scale_beyond_fp16_weight_range_is_reported(dev):
+    """The tensor-core path forms each weight as RNE_fp16(q * s): a scale of
+    10000 with codes of 7 gives 70000, beyond fp16.  Scales above 65504 / 8
+    are reported."""
+    L = Layer.custom(dev, T=40, d=256, E=8, k=2, n=128, group=64, seed=57)
+    _fill(L, "gate_q", 0x77)
+    _fill(L, "gate_s", 10000.0)
+    L.forward()
+    _expect_range_report()
+
+
 def test_token_order_equivariance(dev):
     L = layer_for("default", dev)
     y, ids, _ = L.forward()
@@ -424,3 +480,25 @@ def test_bad_offsets_are_reported_not_used(dev):
     torch.cuda.synchronize()
     assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
     assert bool((h == 7.0).all())                    # nothing was written
+
+
+def test_bounded_waits_give_up_and_leave_the_device_usable(dev):
+    """Waits on conditions nothing satisfies (an mbarrier no thread or copy
+    arrives on, a grid barrier one CTA never reaches) give up after their
+    limit: the kernels return, the time-out is reported, tensor memory held
+    during the wait is released, and the next forward is correct."""
+    out = torch.full((8,), -1, dtype=torch.int32, device=dev)
+    sync = torch.zeros(16, dtype=torch.uint8, device=dev)
+    assert sm.strata_moe_selftest_wait(out, sync) == sm.STRATA_OK
+    torch.cuda.synchronize()
+    o = out.cpu().tolist()
+    assert o[0:4] == [0, 0, 0, 0], o           # warp 0 gave up, the others saw its abort
+    assert 0.9e9 <= o[4] <= 1.9e9, o           # after about the one-second limit
+    assert o[5] == 1, o                        # tensor memory released
+    assert o[6] == 0 and 0.9e9 <= o[7] <= 1.9e9, o
+    assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
+    assert sm.strata_moe_device_status() == sm.STRATA_OK
+    L = Layer.custom(dev, T=40, d=256, E=8, k=2, n=128, group=64, seed=58)
+    y, ids, _ = L.forward()
+    assert_device_ok()
+    _check_forward(L, y, ids, np.arange(40), 2, 64, "after the self-test")
