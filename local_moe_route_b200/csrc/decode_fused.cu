@@ -556,8 +556,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       float4* rp = reinterpret_cast<float4*>(red + (warp * 32 + lane) * 8);
       rp[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
       rp[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-      named_barrier_sync(1, CONS * 32);
-      if (failed || *abort_flag) break;     // uniform: the flag is read after the barrier
+      if (named_barrier_or(1, CONS * 32, failed || *abort_flag)) break;   // all warps alike
       if (threadIdx.x < P2_ROWS * 8) {
         const int r = threadIdx.x >> 3, col = threadIdx.x & 7;
         const int ln = (r & 7) * 4 + (col >> 1), reg = (r >> 3) * 2 + (col & 1);
@@ -643,8 +642,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       // second K half hands its sums to the first (fixed order: first + second)
       float4* rp = reinterpret_cast<float4*>(red + (rg * 32 + lane) * 4);
       if (kh == 1) *rp = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      named_barrier_sync(1, CONS * 32);
-      if (failed || *abort_flag) break;
+      if (named_barrier_or(1, CONS * 32, failed || *abort_flag)) break;   // all warps alike
       if (kh == 0) {
         const float4 o = *rp;
         const float v[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};

@@ -306,8 +306,9 @@ __global__ void __launch_bounds__(dk::THREADS, NMAT == 1 ? 3 : 2)
         if (lane == 0) mbar_arrive(&empty[s]);
       }
       // Every consumer warp reaches the two barriers below, also after a
-      // wait that ran out (which raised abort_flag first): the flag read
-      // between them makes the decision to stop the same in all warps.
+      // wait that ran out (which raised abort_flag first); the first one
+      // reduces the flag over all consumer threads, so the decision to stop
+      // is the same in every warp.
       // The second K half hands its sums to the first (fixed order: first + second).
       if (kh == 1) {
 #pragma unroll
@@ -316,8 +317,7 @@ __global__ void __launch_bounds__(dk::THREADS, NMAT == 1 ? 3 : 2)
           if (NMAT == 2) red[4 + q] = acc[NMAT - 1][q];
         }
       }
-      named_barrier_sync(1, CONSUMERS * 32);
-      failed = *abort_flag != 0;
+      failed = named_barrier_or(1, CONSUMERS * 32, *abort_flag != 0);   // all warps alike
       if (kh == 0) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {

@@ -561,11 +561,11 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     bool ov = false;            // an output of this thread overflowed fp16
     for (int i = 0; i < my_units; ++i) {
       const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
-      if (!mbar_wait_warp(acc_full, i & 1, abort_flag, args.err)) break;
+      const bool got = mbar_wait_warp(acc_full, i & 1, abort_flag, args.err);
       tc_fence_after();
       const int nch = (U.cnt + 31) >> 5;
       const int nout = OP == 0 ? 1 : U.nslots;        // 128-feature slices of output
-      for (int m = 0; m < nout; ++m) {
+      for (int m = 0; m < nout && got; ++m) {
         uint16_t* frow = sStg + (m * BM + q * 32 + lane) * STG_PITCH;
         for (int c = 0; c < nch; ++c) {
           __syncwarp();   // converged before the .sync.aligned TMEM loads
@@ -609,8 +609,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_empty);
-      named_barrier_sync(1, 128);                     // staging tile complete
+      if (got) mbar_arrive(acc_empty);
+      // staging tile complete; a wait that gave up in any epilogue warp ends
+      // the loop in all four alike
+      if (named_barrier_or(1, 128, !got)) break;
       if (et < U.cnt) {
         uint16_t* dst = args.out + (size_t)(U.p0 + et) * N + U.fout[0];
         for (int ch = 0; ch < nout * (BM / 8); ++ch) {
