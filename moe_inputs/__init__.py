@@ -33,7 +33,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_custom", "bf16_bits",
-           "chunk_sizes"]
+           "chunk_sizes", "AttnWorkload", "ATTN_WORKLOADS", "make_attention"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -133,3 +133,50 @@ def make_inputs(w: Workload, T: Optional[int] = None) -> Dict[str, np.ndarray]:
     need one model for several token counts slice ``x`` instead)."""
     return make_custom(w.T if T is None else T, w.d, w.E, w.k, w.n, w.group,
                        w.seed, w.s_lo, w.s_hi, w.zipf, w.x_std, w.wr_std)
+
+
+# --------------------------------------------------------------------------
+# Sparse attention over indexer-selected KV-cache rows (kongchang.com
+# benchmark summary, section "Strata快在哪", attention paragraph: the indexer
+# picks about 2000 positions per query).  The pages give no head counts or
+# head size; the workloads use 32 query heads sharing 4 KV heads (groups of
+# 8), head size 128, a 34,000-token context (the agent prompt of the
+# "为什么预填充比解码更重要" section) and 2048 selected positions per query.
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    name: str
+    T: int          # query tokens
+    L: int          # context length (KV-cache rows)
+    Hq: int         # query heads
+    Hkv: int        # KV heads
+    D: int          # head size
+    P: int          # selected positions per query (index slots)
+    seed: int
+
+
+ATTN_WORKLOADS: Dict[str, AttnWorkload] = {
+    "attn_tiny": AttnWorkload("attn_tiny", T=3, L=300, Hq=8, Hkv=2, D=64, P=64, seed=11),
+    "attn_decode1": AttnWorkload("attn_decode1", T=1, L=34000, Hq=32, Hkv=4, D=128, P=2048,
+                                 seed=12),
+    "attn_verify4": AttnWorkload("attn_verify4", T=4, L=34000, Hq=32, Hkv=4, D=128, P=2048,
+                                 seed=13),
+}
+
+
+def make_attention(T: int, L: int, Hq: int, Hkv: int, D: int, P: int, seed: int,
+                   n_valid: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """q [T][Hq][D], k / v [L][Hkv][D] as bf16 bits (values ~N(0,1)), idx
+    [T][P] int32: per query a seeded draw of distinct positions in [0, L),
+    ascending; with n_valid[t] < P the remaining slots hold -1.
+    Draw order: q, k, v, then the positions of each query."""
+    rng = np.random.default_rng(seed)
+    out: Dict[str, np.ndarray] = {}
+    out["q"] = bf16_bits(rng.standard_normal((T, Hq, D), dtype=np.float32))
+    out["k"] = bf16_bits(rng.standard_normal((L, Hkv, D), dtype=np.float32))
+    out["v"] = bf16_bits(rng.standard_normal((L, Hkv, D), dtype=np.float32))
+    idx = np.full((T, P), -1, np.int32)
+    for t in range(T):
+        m = P if n_valid is None else int(n_valid[t])
+        idx[t, :m] = np.sort(rng.choice(L, size=m, replace=False)).astype(np.int32)
+    out["idx"] = idx
+    return out
