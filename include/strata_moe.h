@@ -259,6 +259,32 @@ STRATA_API strata_status_t strata_moe_gather_rows(const uint16_t* src, const int
                                        int32_t src_rows, int32_t rows, int32_t width,
                                        uint16_t* dst, strata_stream_t stream);
 
+/* Attention over the KV-cache rows an indexer selected.  The pages' model
+ * picks about 2000 positions per query with an indexer, and Strata's kernel
+ * reads only the selected KV-cache rows where llama.cpp builds a full mask
+ * and runs dense flash attention (kongchang.com "两天移植，预填充提速8倍：
+ * Strata引擎实测", section "Strata快在哪", attention paragraph).  For query
+ * token t and query head h, with KV head hk = h / (Hq / Hkv):
+ *   o[t][h] = sum_p softmax_p(scale * q[t][h] . K[p][hk]) V[p][hk],
+ *             p over idx[t][0..P) with slots of -1 unused
+ *   T   query tokens            L    KV-cache rows
+ *   Hq  query heads             Hkv  KV heads (Hq % Hkv == 0, Hq / Hkv <= 16)
+ *   D   head size (64 or 128)   P    index slots per query (<= 65536)
+ *   q [T][Hq][D] bf16, k_cache / v_cache [L][Hkv][D] bf16, idx [T][P] int32,
+ *   out [T][Hq][D] bf16; scale <= 0 means 1 / sqrt(D)
+ * Scores, softmax and the weighted sum in fp32; one rounding to bf16.  A
+ * query with no selected row gets zeros.  An index >= L is reported through
+ * strata_moe_device_status() and skipped.  The pages fix no head counts,
+ * head size or index format; these are this library's readings. */
+typedef struct {
+  int32_t T, L, Hq, Hkv, D, P;
+} strata_attn_dims_t;
+STRATA_API size_t strata_sparse_attention_workspace_bytes(strata_attn_dims_t dims);
+STRATA_API strata_status_t strata_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
+                                        const uint16_t* v_cache, const int32_t* idx,
+                                        strata_attn_dims_t dims, float scale, uint16_t* out,
+                                        void* ws, size_t ws_bytes, strata_stream_t stream);
+
 /* Synchronises `stream`, then reports (and clears) the device-side check word
  * of the current device: STRATA_OK, or STRATA_ERR_DEVICE_CHECK when a kernel
  * since the last call recorded an out-of-range index or a bounded wait that

@@ -23,7 +23,8 @@ __all__ = [
     "strata_moe_permute", "strata_moe_permute_static", "STRATA_PERMUTE_STATIC_SCRATCH_INTS",
     "strata_moe_expert_gemm_q4", "strata_moe_combine",
     "strata_moe_forward", "strata_moe_device_status", "strata_moe_selftest_wait",
-    "strata_moe_gather_rows", "workspace",
+    "strata_moe_gather_rows", "workspace", "AttnDims", "strata_sparse_attention",
+    "strata_sparse_attention_workspace_bytes", "attention_workspace",
 ]
 
 STRATA_OK = 0
@@ -58,6 +59,19 @@ class Dims(ctypes.Structure):
         if isinstance(dims, dict):
             return cls(int(dims["T"]), int(dims["d"]), int(dims["E"]), int(dims["k"]),
                        int(dims["n"]), int(dims["group"]))
+        return cls(*[int(v) for v in dims])
+
+
+class AttnDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("L", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32), ("P", ctypes.c_int32)]
+
+    @classmethod
+    def of(cls, dims: Any) -> "AttnDims":
+        if isinstance(dims, cls):
+            return dims
+        if isinstance(dims, dict):
+            return cls(*[int(dims[k]) for k in ("T", "L", "Hq", "Hkv", "D", "P")])
         return cls(*[int(v) for v in dims])
 
 
@@ -113,6 +127,11 @@ def lib() -> ctypes.CDLL:
     i32 = ctypes.c_int32
     L.strata_moe_gather_rows.argtypes = [vp, vp, i32, i32, i32, vp, vp]
     L.strata_moe_gather_rows.restype = st
+    L.strata_sparse_attention_workspace_bytes.argtypes = [AttnDims]
+    L.strata_sparse_attention_workspace_bytes.restype = sz
+    L.strata_sparse_attention.argtypes = [vp, vp, vp, vp, AttnDims, ctypes.c_float, vp, vp, sz,
+                                          vp]
+    L.strata_sparse_attention.restype = st
     _lib = L
     return L
 
@@ -211,6 +230,26 @@ def strata_moe_selftest_wait(out, sync_ws, stream=None) -> int:
 def strata_moe_gather_rows(src, index, src_rows, rows, width, dst, stream=None) -> int:
     return lib().strata_moe_gather_rows(_ptr(src), _ptr(index), int(src_rows), int(rows),
                                         int(width), _ptr(dst), _stream(stream))
+
+
+def strata_sparse_attention_workspace_bytes(dims) -> int:
+    return int(lib().strata_sparse_attention_workspace_bytes(AttnDims.of(dims)))
+
+
+def strata_sparse_attention(q, k_cache, v_cache, idx, dims, scale, out, ws=None, ws_bytes=None,
+                            stream=None) -> int:
+    return lib().strata_sparse_attention(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx), AttnDims.of(dims), float(scale),
+        _ptr(out), _ptr(ws), _nbytes(ws) if ws_bytes is None else int(ws_bytes), _stream(stream))
+
+
+def attention_workspace(dims, device="cuda"):
+    """A torch uint8 buffer of strata_sparse_attention_workspace_bytes(dims) bytes."""
+    import torch
+    n = strata_sparse_attention_workspace_bytes(dims)
+    if n == 0:
+        raise StrataError(STRATA_ERR_INVALID_ARG, "attention workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def workspace(dims, device="cuda"):

@@ -455,6 +455,38 @@ strata_status_t strata_moe_gather_rows(const uint16_t* src, const int32_t* index
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static strata_status_t check_attn_dims(const strata_attn_dims_t& a) {
+  if (a.T < 0 || a.L <= 0 || a.Hq <= 0 || a.Hkv <= 0 || a.P <= 0 || a.Hq % a.Hkv)
+    return STRATA_ERR_INVALID_ARG;
+  if ((a.D != 64 && a.D != 128) || a.Hq / a.Hkv > 16 || a.P > 65536)
+    return STRATA_ERR_UNSUPPORTED;
+  return STRATA_OK;
+}
+
+size_t strata_sparse_attention_workspace_bytes(strata_attn_dims_t dims) {
+  if (check_attn_dims(dims) != STRATA_OK) return 0;
+  return sparse_attn_scratch(dims.T, dims.Hq, dims.P, dims.D) + 256;
+}
+
+strata_status_t strata_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
+                                        const uint16_t* v_cache, const int32_t* idx,
+                                        strata_attn_dims_t dims, float scale, uint16_t* out,
+                                        void* ws, size_t ws_bytes, strata_stream_t stream) {
+  strata_status_t st = check_attn_dims(dims);
+  if (st != STRATA_OK) return st;
+  if (dims.T == 0) return STRATA_OK;
+  if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(idx) || !ok_ptr(out))
+    return STRATA_ERR_INVALID_ARG;
+  if (!ok_ptr(ws) || ws_bytes < sparse_attn_scratch(dims.T, dims.Hq, dims.P, dims.D))
+    return STRATA_ERR_WORKSPACE;
+  unsigned* err = check_word_ptr();
+  if (!err) return STRATA_ERR_CUDA;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)dims.D);
+  return cuda_status(launch_sparse_attn(q, k_cache, v_cache, idx, dims.T, dims.L, dims.Hq,
+                                        dims.Hkv, dims.D, dims.P, scale, out, ws, err,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 strata_status_t strata_moe_device_status(strata_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return STRATA_ERR_CUDA;

@@ -99,4 +99,11 @@ cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* index, int sr
                                int rows, int width, uint16_t* dst, unsigned* err,
                                cudaStream_t s);
 
+// ---- attention over indexer-selected KV rows
+size_t sparse_attn_scratch(int T, int Hq, int P, int D);
+cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                               const int32_t* idx, int T, int L, int Hq, int Hkv, int D, int P,
+                               float scale, uint16_t* out, void* ws, unsigned* err,
+                               cudaStream_t s);
+
 }  // namespace strata

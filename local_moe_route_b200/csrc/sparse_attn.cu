@@ -1,0 +1,180 @@
+// sparse_attn.cu -- attention over the KV-cache rows an indexer selected.
+//
+// The pages' model uses sparse attention: an indexer picks about 2000
+// positions for every query, and Strata's own kernel reads only the
+// selected KV-cache rows where llama.cpp builds a full mask and runs dense
+// flash attention (kongchang.com "两天移植，预填充提速8倍：Strata引擎实测",
+// section "Strata快在哪", attention paragraph).  Per query token t and query
+// head h (KV head hk = h / (Hq / Hkv)):
+//   o[t][h] = softmax_p( scale * q[t][h] . K[p][hk] ) . V[p][hk],  p in idx[t]
+// with idx slots of -1 unused.
+//
+// Small query batches (decode, speculative verify) are bound by the bytes of
+// the selected rows, 2 * Hkv * D * 2 bytes per position per query.  Two
+// kernels, split-K style:
+//   1. one CTA per (query, KV head, slice of 128 index slots): every thread
+//      takes one slot, reads its K row (16-byte loads) and forms the scores of
+//      the G query heads that share the KV head; the slice's softmax maximum
+//      and sum per head go to shared memory; then thread d accumulates
+//      sum_p exp(s - m) V[p][d] over the slice (V rows read whole by the
+//      block, 256 bytes per row), fp32;
+//   2. one CTA per (query, head) rescales and adds the slices' partial sums
+//      (max-subtracted exponentials, fixed order) and rounds to bf16.
+#include "common.cuh"
+#include "internal.h"
+
+namespace strata {
+
+namespace sa {
+constexpr int SLICE = 128;     // index slots per CTA (one per thread)
+constexpr int THREADS = 128;
+constexpr int MAXG = 16;       // query heads per KV head
+}  // namespace sa
+
+template <int D>
+__global__ void __launch_bounds__(sa::THREADS)
+    sparse_attn_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc,
+                             const uint16_t* __restrict__ vc, const int32_t* __restrict__ idx,
+                             int L, int Hq, int Hkv, int P, int nsplit, float scale,
+                             float* __restrict__ part_o, float* __restrict__ part_ml,
+                             unsigned* err) {
+  using namespace sa;
+  const int split = blockIdx.x, hk = blockIdx.y, t = blockIdx.z;
+  const int G = Hq / Hkv;
+  __shared__ float qs[MAXG][D];
+  __shared__ float ws[MAXG][SLICE];          // scores, then exp(s - m)
+  __shared__ int rows[SLICE];
+  __shared__ float mx[MAXG], sm[MAXG];
+  const int th = threadIdx.x;
+  for (int i = th; i < G * D; i += THREADS) {
+    const int g = i / D, dd = i % D;
+    qs[g][dd] = __uint_as_float((uint32_t)q[((size_t)t * Hq + hk * G + g) * D + dd] << 16) * scale;
+  }
+  const int slot = split * SLICE + th;
+  int p = -1;
+  if (slot < P) {
+    p = idx[(size_t)t * P + slot];
+    if (p >= L) {
+      atomicOr(err, kErrIndex);
+      p = -1;
+    }
+  }
+  rows[th] = p;
+  __syncthreads();
+  // scores of this thread's position for the G heads
+  float s[MAXG];
+#pragma unroll
+  for (int g = 0; g < MAXG; ++g) s[g] = 0.f;
+  if (p >= 0) {
+    const uint4* kr = reinterpret_cast<const uint4*>(kc + ((size_t)p * Hkv + hk) * D);
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = __ldg(kr + c);
+      const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                          bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+      for (int g = 0; g < MAXG; ++g) {
+        if (g < G) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) s[g] = fmaf(qs[g][8 * c + j], e[j], s[g]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < MAXG; ++g)
+    if (g < G) ws[g][th] = p >= 0 ? s[g] : -INFINITY;
+  __syncthreads();
+  // per head: maximum and sum of exp(s - m) over the slice (warp g % 4 takes heads g)
+  const int warp = th >> 5, lane = th & 31;
+  for (int g = warp; g < G; g += THREADS / 32) {
+    float m = -INFINITY;
+    for (int i = lane; i < SLICE; i += 32) m = fmaxf(m, ws[g][i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float l = 0.f;
+    for (int i = lane; i < SLICE; i += 32) {
+      const float e = ws[g][i] == -INFINITY ? 0.f : __expf(ws[g][i] - m);
+      ws[g][i] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (lane == 0) {
+      mx[g] = m;
+      sm[g] = l;
+    }
+  }
+  __syncthreads();
+  // o[g][d] = sum_p e[g][p] V[p][d]; thread = feature d (D <= 128 threads)
+  if (th < D) {
+    float o[MAXG];
+#pragma unroll
+    for (int g = 0; g < MAXG; ++g) o[g] = 0.f;
+    for (int i = 0; i < SLICE; ++i) {
+      const int pr = rows[i];
+      if (pr < 0) continue;
+      const float v = __uint_as_float((uint32_t)__ldg(vc + ((size_t)pr * Hkv + hk) * D + th) << 16);
+#pragma unroll
+      for (int g = 0; g < MAXG; ++g)
+        if (g < G) o[g] = fmaf(ws[g][i], v, o[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < MAXG; ++g)
+      if (g < G) part_o[(((size_t)t * Hq + hk * G + g) * nsplit + split) * D + th] = o[g];
+  }
+  if (th < G) {
+    const size_t b = (((size_t)t * Hq + hk * G + th) * nsplit + split) * 2;
+    part_ml[b] = mx[th];
+    part_ml[b + 1] = sm[th];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D)
+    sparse_attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                               int nsplit, uint16_t* __restrict__ out) {
+  const int th = threadIdx.x;
+  const size_t th_h = blockIdx.x;            // t * Hq + h
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part_ml[(th_h * nsplit + s) * 2]);
+  float num = 0.f, den = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float m = part_ml[(th_h * nsplit + s) * 2];
+      if (m == -INFINITY) continue;
+      const float f = __expf(m - M);
+      den = fmaf(f, part_ml[(th_h * nsplit + s) * 2 + 1], den);
+      num = fmaf(f, part_o[(th_h * nsplit + s) * D + th], num);
+    }
+  }
+  const float o = den > 0.f ? num / den : 0.f;
+  out[th_h * D + th] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+}
+
+size_t sparse_attn_scratch(int T, int Hq, int P, int D) {
+  const int nsplit = (P + sa::SLICE - 1) / sa::SLICE;
+  return ((size_t)T * Hq * nsplit * (D + 2) * 4 + 255) & ~size_t(255);
+}
+
+cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                               const int32_t* idx, int T, int L, int Hq, int Hkv, int D, int P,
+                               float scale, uint16_t* out, void* ws, unsigned* err,
+                               cudaStream_t s) {
+  const int nsplit = (P + sa::SLICE - 1) / sa::SLICE;
+  float* part_o = static_cast<float*>(ws);
+  float* part_ml = part_o + (size_t)T * Hq * nsplit * D;
+  const dim3 grid(nsplit, Hkv, T);
+  if (D == 128) {
+    sparse_attn_split_kernel<128><<<grid, sa::THREADS, 0, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
+                                                               nsplit, scale, part_o, part_ml, err);
+    sparse_attn_combine_kernel<128><<<T * Hq, 128, 0, s>>>(part_o, part_ml, nsplit, out);
+  } else {
+    sparse_attn_split_kernel<64><<<grid, sa::THREADS, 0, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
+                                                              nsplit, scale, part_o, part_ml, err);
+    sparse_attn_combine_kernel<64><<<T * Hq, 64, 0, s>>>(part_o, part_ml, nsplit, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace strata

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
         "strata_moe_permute", "strata_moe_permute_static", "strata_moe_expert_gemm_q4",
         "strata_moe_combine",
         "strata_moe_forward", "strata_moe_device_status", "strata_moe_selftest_wait",
-        "strata_moe_gather_rows"}
+        "strata_moe_gather_rows", "strata_sparse_attention",
+        "strata_sparse_attention_workspace_bytes"}
 
 
 def test_library_exports_every_declared_symbol():
