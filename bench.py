@@ -42,7 +42,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import WORKLOADS, Workload, chunk_sizes, make_inputs  # noqa: E402
+from moe_inputs import (ATTN_WORKLOADS, WORKLOADS, Workload, chunk_sizes,  # noqa: E402
+                        make_attention, make_inputs)
 
 METRIC = "MoE-layer tokens/s at T=6144, 512 experts top-10; % of tensor/HBM roofline"
 # Sources each profiled kernel is built from: its DRAM counters in
@@ -502,6 +503,8 @@ def run_ours(args, wl):
         for name in ("verify4", "decode1", "default", "skewed"):
             if name != wl.name:
                 out["secondary"][name] = run_secondary(sm, dev, WORKLOADS[name], args)
+        for name in ("attn_verify4", "attn_decode1"):
+            out["secondary"][name] = run_secondary_attention(sm, dev, ATTN_WORKLOADS[name], args)
     if world == 1 and args.sustain_s > 0:
         out["sustained"] = run_sustained(R, args.sustain_s, dev, tf_burst, tf_sus, peak_kind)
     if not args.no_cpu_baseline:
@@ -675,6 +678,50 @@ def run_secondary(sm, dev, wl, args):
     gc.collect()
     torch.cuda.empty_cache()
     return res
+
+
+def run_secondary_attention(sm, dev, aw, args):
+    """Attention over the indexer-selected KV rows of a 34,000-token cache:
+    device time of strata_sparse_attention (two kernels), L2 overwritten
+    before every call, HBM roofline over the selected K and V rows."""
+    import torch
+    hbm, _, _, peak_kind = measured_peaks()
+    a = make_attention(aw.T, aw.L, aw.Hq, aw.Hkv, aw.D, aw.P, aw.seed)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    q, k, v, idx = t(a["q"]), t(a["k"]), t(a["v"]), t(a["idx"])
+    dims = dict(T=aw.T, L=aw.L, Hq=aw.Hq, Hkv=aw.Hkv, D=aw.D, P=aw.P)
+    out = torch.empty((aw.T, aw.Hq, aw.D), dtype=torch.bfloat16, device=dev)
+    ws = sm.attention_workspace(dims, dev)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        sm.check(sm.strata_sparse_attention(q, k, v, idx, dims, 0.0, out, ws, stream=stream))
+
+    for _ in range(args.warmup):
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.secondary_steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert sm.strata_moe_device_status() == sm.STRATA_OK
+    ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    med = statistics.median(ms)
+    valid = int(np.sum(a["idx"] >= 0))
+    rows_bytes = valid * aw.Hkv * aw.D * 2 * 2            # selected K and V rows
+    bytes_ = rows_bytes + a["idx"].nbytes + 2 * aw.T * aw.Hq * aw.D * 2
+    return {"T": aw.T, "L": aw.L, "Hq": aw.Hq, "Hkv": aw.Hkv, "D": aw.D, "P": aw.P,
+            "ms_per_call": round(med, 5), "steps": len(ms),
+            "queries_per_s": round(aw.T / (med / 1e3), 1),
+            "l2": "flushed (256 MB write) before each call",
+            "roofline": roof(bytes_ / (med / 1e3) / 1e9, hbm, "GB/s", "hbm",
+                             f"{peak_kind} copy bandwidth", bytes_per_call=bytes_,
+                             kernel="sparse_attn_split_kernel + sparse_attn_combine_kernel"),
+            "dense_cache_bytes": 2 * aw.L * aw.Hkv * aw.D * 2}
 
 
 # --------------------------------------------------------------------------- sustained
