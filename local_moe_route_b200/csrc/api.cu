@@ -140,10 +140,10 @@ Schedule schedule_at(uint8_t* ws, const SchedRegions& r) {
   s.n_active = reinterpret_cast<int32_t*>(ws + r.n_active.off);
   return s;
 }
-// x in fp16, token order [T][d]: the tensor-core gate/up path (batches above
-// the streaming threshold) gathers its B rows from it.
+// fp16 rows of x in grouped order [T*k][d], the B operand of the tensor-core
+// gate/up path (batches above the streaming threshold).
 size_t x16_bytes(const strata_moe_dims_t& d) {
-  return d.T > kStreamMaxTokens ? (size_t)d.T * d.d * 2 : 0;
+  return d.T > kStreamMaxTokens ? (size_t)d.T * d.k * d.d * 2 : 0;
 }
 size_t gemm_scratch(const strata_moe_dims_t& d) {
   Layout L;

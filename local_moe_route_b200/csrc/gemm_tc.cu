@@ -24,12 +24,14 @@
 //   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
 //                swizzle) into an 8-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
-//   warp 2       token rows into a 4-deep ring: the down projection reads h,
-//                whose rows are already grouped by expert, as one TMA tile of
-//                128 rows per stage; gate/up gathers its rows x16[sorted_token[p]]
-//                from an fp16 copy of x in token order (written once per call)
-//                with tile::gather4 copies, four rows each, issued by the 32
-//                lanes of the warp, so x is never copied in grouped order.
+//   warp 2       token rows into a 4-deep ring, one TMA tile of 128 rows per
+//                stage: the down projection reads h, whose rows are already
+//                grouped by expert; for gate/up a pre-pass writes the fp16 rows
+//                of x in grouped order (x[sorted_token[p]]), so both operands
+//                of every stage arrive by TMA.  (Gathering the rows from a
+//                token-order copy with tile::gather4 copies instead, 32 per
+//                stage, left the MMA waiting on them 64% of the time and
+//                doubled the kernel's time at T = 6144.)
 //   warps 3-10   two dequantising warpgroups taking alternate stages; thread
 //                = weight row; fp16 pairs go to TMEM with tcgen05.st; each
 //                thread loads its row's group scales one block of groups
@@ -39,8 +41,8 @@
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/128, four A
 // stages of 64 columns (32 per slot) at 256..511.
 //
-// Operands are fp16 (kind::f16): x is copied to fp16 once per call (exact for
-// |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
+// Operands are fp16 (kind::f16): x rows are copied to fp16 in grouped order
+// once per call (exact for |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
 // keeps q * s to 2^-11, where bf16 weights (2^-8) would use up most of the
 // layer's error budget.  Dequantisation: the nibble with its sign bit flipped
 // goes into the mantissa of 1024.0 (giving 1032 + q), one fma subtracts 1032
@@ -178,35 +180,46 @@ __device__ __forceinline__ void dequant8_interleaved(uint32_t w, uint32_t sc2, u
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[3]) : "r"(q3), "r"(sc2));
 }
 
-// Gate/up B operand: x16 = fp16(x) for the T token rows, with K interleaved
-// within each group of 8 (0, 4, 1, 5, 2, 6, 3, 7) to match
-// dequant8_interleaved.  Values beyond the fp16 range become +-inf and are
-// reported as kErrRange.
+// Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]) for the S grouped rows,
+// with K interleaved within each group of 8 (0, 4, 1, 5, 2, 6, 3, 7) to match
+// dequant8_interleaved.  Out-of-range token indices are reported (kErrIndex)
+// and read row 0; values beyond the fp16 range become +-inf and are reported
+// as kErrRange.
 __global__ void __launch_bounds__(256)
-    convert_x_f16_kernel(const uint16_t* __restrict__ x, long chunks,
-                         uint16_t* __restrict__ x16, unsigned* err) {
-  // 16-byte chunks (8 values, one K group of 8) in a grid-stride loop
-  bool over = false;
-  const uint4* src = reinterpret_cast<const uint4*>(x);
-  uint4* dst = reinterpret_cast<uint4*>(x16);
-  for (long c = blockIdx.x * (long)blockDim.x + threadIdx.x; c < chunks;
-       c += (long)gridDim.x * blockDim.x) {
-    const uint4 v = __ldg(src + c);
-    float e[8];
-    e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
-    e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
+    gather_rows_f16_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
+                           int T, int d, int S, uint16_t* __restrict__ xs, unsigned* err) {
+  // one warp per grouped row; lane l converts 16-byte chunks l, l + 32, ...
+  const int lane = threadIdx.x & 31;
+  const int cpr = d / 8;                      // 16-byte chunks per row
+  bool over = false, bad = false;
+  for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < S; p += gridDim.x * 8) {
+    int t = sorted_token[p];
+    if ((unsigned)t >= (unsigned)T) {
+      bad = true;
+      t = 0;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * d);
+#pragma unroll 2
+    for (int c = lane; c < cpr; c += 32) {
+      const uint4 v = __ldg(src + c);
+      float e[8];
+      e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
+      e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
-    // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
-    // weight dequantisation produces)
-    uint4 o;
-    o.x = pack_f16x2(e[0], e[4]);
-    o.y = pack_f16x2(e[1], e[5]);
-    o.z = pack_f16x2(e[2], e[6]);
-    o.w = pack_f16x2(e[3], e[7]);
-    dst[c] = o;
+      for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
+      // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
+      // weight dequantisation produces)
+      uint4 o;
+      o.x = pack_f16x2(e[0], e[4]);
+      o.y = pack_f16x2(e[1], e[5]);
+      o.z = pack_f16x2(e[2], e[6]);
+      o.w = pack_f16x2(e[3], e[7]);
+      dst[c] = o;
+    }
   }
   if (over) atomicOr(err, kErrRange);
+  if (bad) atomicOr(err, kErrIndex);
 }
 
 template <int OP, bool ILV>
@@ -277,7 +290,6 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     // -------------------------------------------------------------- TMA producer
     if (lane == 0) {
       const CUtensorMap* map_slot1 = OP == 0 ? &map_q1 : &map_q0;
-      const uint64_t once = l2_policy_evict_first();   // every weight is read once
       uint32_t g = 0;
       bool stop = false;
       for (int i = 0; i < my_units && !stop; ++i) {
@@ -290,53 +302,17 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&raw_full[s], 2 * RAW_BYTES);
-          tma_load_2d_hint(sRaw + (s * 2 + 0) * RAW_BYTES, &map_q0, kb * (BK / 2), U.wrow[0],
-                           &raw_full[s], once);
-          tma_load_2d_hint(sRaw + (s * 2 + 1) * RAW_BYTES, map_slot1, kb * (BK / 2), U.wrow[1],
-                           &raw_full[s], once);
+          tma_load_2d(sRaw + (s * 2 + 0) * RAW_BYTES, &map_q0, kb * (BK / 2), U.wrow[0],
+                      &raw_full[s]);
+          tma_load_2d(sRaw + (s * 2 + 1) * RAW_BYTES, map_slot1, kb * (BK / 2), U.wrow[1],
+                      &raw_full[s]);
         }
       }
     }
-  } else if (warp == W_BTMA && OP == 0) {
-    // -------------------------------------------------------------- token rows (B), gate/up
-    // The unit's rows are the tokens sorted_token[p0 .. p0 + cnt) of x16.
-    // Lane l gathers tile rows 4l .. 4l + 3 with one gather4 copy per stage;
-    // rows past the unit repeat its last token (their MMA columns are not
-    // used), rows past the last group of four are not loaded.
-    uint32_t g = 0;
-    bool stop = false, bad = false;
-    for (int i = 0; i < my_units && !stop; ++i) {
-      const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
-      int tok[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = min(4 * lane + j, U.cnt - 1);
-        int t = args.sorted_token[U.p0 + r];
-        if ((unsigned)t >= (unsigned)args.a_rows) {
-          bad = true;
-          t = 0;
-        }
-        tok[j] = t;
-      }
-      const int ng = (U.cnt + 3) >> 2;           // gather4 copies per stage
-      for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % B_ST;
-        if (g >= (uint32_t)B_ST &&
-            !mbar_wait_warp(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
-          stop = true;
-          break;
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&b_full[s], (uint32_t)ng * 4u * (BK * 2));
-        __syncwarp();
-        if (lane < ng) tma_gather4(sB + s * B_BYTES + lane * 4 * (BK * 2), &map_b, kb * BK, tok,
-                                   &b_full[s]);
-      }
-    }
-    if (bad) atomicOr(args.err, kErrIndex);
   } else if (warp == W_BTMA) {
-    // -------------------------------------------------------------- token rows (B), down
-    // one TMA tile of 128 grouped rows of h per stage (rows past the unit
-    // belong to other units or lie beyond S; the MMA reads only nrows of them)
+    // -------------------------------------------------------------- token rows (B)
+    // one TMA tile of 128 grouped rows per stage (rows past the unit belong
+    // to other units or lie beyond S; the MMA reads only nrows of them)
     if (lane == 0) {
       uint32_t g = 0;
       bool stop = false;
@@ -657,12 +633,11 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   m1 = m0;
-  // B rows: gate/up gathers rows of the fp16 copy of x [T][K] four at a time
-  // (one-row box); down reads h [S][K] in 128-row tiles
+  // B rows: grouped fp16 rows [S][K] (the gathered copy of x, or h)
   CUtensorMap mb;
   const uint16_t* brows = OP == 0 ? p.a16 : p.a;
-  if (encode_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, brows, p.K, OP == 0 ? p.T : p.S,
-                     (uint64_t)p.K * 2, tc::BK, OP == 0 ? 1 : tc::NT, CU_TENSOR_MAP_SWIZZLE_128B,
+  if (encode_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, brows, p.K, p.S, (uint64_t)p.K * 2,
+                     tc::BK, tc::NT, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (OP == 0 &&
@@ -677,11 +652,11 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   }
   const int num_sms = sm_count();
   if (OP == 0) {
-    // the gate/up B operand: x in fp16, token order
-    const long chunks = (long)p.T * p.K / 8;
-    long blocks = (chunks + 255) / 256;
-    if (blocks > 8L * num_sms) blocks = 8L * num_sms;
-    convert_x_f16_kernel<<<(int)blocks, 256, 0, s>>>(p.a, chunks, p.a16, p.err);
+    // the gate/up B operand: fp16 rows of x in grouped order
+    long blocks = (p.S + 7) / 8;                     // 8 rows (warps) per block
+    if (blocks > 16L * num_sms) blocks = 16L * num_sms;
+    gather_rows_f16_kernel<<<(int)blocks, 256, 0, s>>>(p.a, p.sorted_token, p.T, p.K, p.S, p.a16,
+                                                       p.err);
   }
   TcArgs a;
   a.a = brows;

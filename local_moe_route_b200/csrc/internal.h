@@ -64,7 +64,7 @@ struct GemmProblem {
   const uint8_t* q0; const uint16_t* s0;  // gate (or down)
   const uint8_t* q1; const uint16_t* s1;  // up (gate/up only)
   const float* row_scale;       // down only, nullable
-  uint16_t* a16;                // scratch [T][d]: x in fp16, token order (TC gate/up)
+  uint16_t* a16;                // scratch [T*k][d]: fp16 x rows in grouped order (TC gate/up)
   uint16_t* out;
   int T, S, E, K, N, G;         // K reduction dim, N output features
   // Tensor-core path only, set by the fused forward: h travels between the

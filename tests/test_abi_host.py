@@ -61,8 +61,8 @@ LARGE = dict(T=6144, d=4096, E=512, k=10, n=1024, group=64)
 def test_workspace_bytes():
     n = sm.strata_moe_workspace_bytes(LARGE)
     S = 6144 * 10
-    # at least the fp16 buffers: x in token order [T][d], h [S][n], rows [S][d]
-    rows = 6144 * 4096 * 2 + S * 1024 * 2 + S * 4096 * 2
+    # at least the per-row fp16 buffers: grouped x [S][d], h [S][n], rows [S][d]
+    rows = S * 4096 * 2 + S * 1024 * 2 + S * 4096 * 2
     assert n >= rows
     assert n < rows + 64 * 2 ** 20
     assert n % 256 == 0
