@@ -150,8 +150,9 @@ def device_layer(inp, dev):
 def fused_decode(T, d, E, k, n, group):
     """Whether strata_moe_forward runs the batch as one persistent launch
     (mirrors the library's rule for batches of at most four tokens)."""
-    if not (1 <= T <= 4 and k <= 32 and E <= 1024 and group in (32, 64, 128)
-            and d % 1024 == 0 and n % 256 == 0):
+    if not (1 <= T <= 4 and k <= 32 and E <= 1024 and E % 8 == 0 and group in (32, 64, 128)
+            and d % 1024 == 0 and d <= 4096 and n % 256 == 0
+            and (n // group) % 8 == 0 and n // group <= 64):
         return False
     xbytes = (T * (d + 8) * 2 + 1023) // 1024 * 1024
     smem = 3 * 16384 + xbytes + 8 * 32 * 8 * 4 + 128 + (2 * 128 + 4 * 1024 + 1 + 2 * 128 + 64) * 4

@@ -10,7 +10,7 @@
 // launch: the CTAs stay resident (cooperative launch, two per SM) and pass
 // through five phases separated by grid-wide barriers with bounded waits:
 //
-//   P0  router partial logits (K in 512-row slices x 16 experts per item);
+//   P0  router partial logits (items of 512 rows of W_r x 64 experts);
 //       every CTA also converts x of all tokens to fp16 in shared memory;
 //   --- grid barrier
 //   P1  every CTA sums the partials, picks each token's top k (exact ties to
@@ -45,13 +45,20 @@ constexpr int MAXT = 4;                   // tokens per batch on this path
 constexpr int CONS = 8;                   // consumer warps
 constexpr int THREADS = (CONS + 1) * 32;  // + one producer warp
 constexpr int ST = 3;                     // ring stages
-constexpr int SLOT = 16384;               // bytes per ring stage
+// A ring stage: gate/up: 16 rows x 1024 K of both matrices (16 KB) and their
+// scales (16 rows x 1024 / G groups each, at most 2 KB); down: 64 rows x
+// 256 K (8 KB), the expert's h rows (2 KB) and the unit's scale rows
+// (64 rows x n / G groups, at most 4 KB).
+constexpr int SLOT = 18432;               // bytes per ring stage
+constexpr int P2_SC = 16384;              // offset of the gate/up scales in a stage
+constexpr int P3_H = 8192, P3_SC = 10240; // offsets of h and of the down scales
 constexpr int P2_ROWS = 16;               // gate/up unit: 16 rows, K split 8 ways
 constexpr int P2_KST = 1024;              // gate/up K per stage
 constexpr int P3_ROWS = 64;               // down unit: 4 row groups x 2 K halves
 constexpr int P3_KST = 256;               // down K per stage
 constexpr int P0_RS = 512;                // router rows per item
-constexpr int P0_EC = 16;                 // router experts per item
+constexpr int P0_MAXKS = 8;               // router K slices (d <= 4096)
+constexpr int XPT = 8;                    // 16-byte chunks of x per thread (T * d <= 8 * 8 * THREADS)
 constexpr int MAXE = 1024, MAXK = 32;
 constexpr int MAXS = MAXT * MAXK;
 
@@ -68,9 +75,9 @@ struct Smem {
     s.red = s.x + xb;                            // [8 warps][32 lanes][8] fp32
     s.bars = s.red + CONS * 32 * 8 * 4;
     s.route = s.bars + 128;
-    // ids, w [MAXS]; counts, active, pos [MAXE]; offsets [MAXE + 1]; rowtok,
-    // slotrow [MAXS]; misc [64]
-    s.total = s.route + (2 * MAXS + 3 * MAXE + MAXE + 1 + 2 * MAXS + 64) * 4;
+    // ids, w [MAXS]; counts, active [MAXE]; offsets [MAXE + 1]; rowtok,
+    // slotrow [MAXS]; misc [64]  (the scan scratch `pos` lives in the ring)
+    s.total = s.route + (2 * MAXS + 2 * MAXE + MAXE + 1 + 2 * MAXS + 64) * 4;
     return s;
   }
 };
@@ -156,40 +163,68 @@ __device__ int df_block_scan(int* v, int n, int* tmp) {
 }
 
 // ---------------------------------------------------------------------------
-// P0: partial router logits.  Item = (16 experts, 512 rows of W_r); thread
-// (row group rg = th / 16, expert e0 + th % 16) sums every 18th row, then the
-// 18 row groups are added in a fixed order.  red: >= 18 * 4 * 16 floats.
-__device__ void df_router_partials(const FusedArgs& a, float* red) {
+// P0: partial router logits.  Item = (512 rows of W_r, 64 experts): thread
+// (row group rr = th / 8 of 32, 16-byte chunk c = th % 8 of 8 experts) loads
+// the chunk of rows rr, rr + 32, ... (16 rows) all at once, multiplies them
+// by x of those rows (staged per item in shared memory as fp32) and the 32
+// row groups are added in a fixed order.  Uses threads 0..255.
+//   scratch: >= 32 * MAXT * 64 + MAXT * 512 floats
+__device__ void df_router_partials(const FusedArgs& a, float* scratch) {
   using namespace df;
-  const int th = threadIdx.x, el = th & 15, rg = th >> 4;   // rg < 18
-  const int nec = (a.E + P0_EC - 1) / P0_EC, nks = a.d / P0_RS;
-  for (int item = blockIdx.x; item < nec * nks; item += gridDim.x) {
-    const int ec = item % nec, ks = item / nec;
-    const int e = ec * P0_EC + el;
-    float acc[MAXT];
-#pragma unroll
-    for (int t = 0; t < MAXT; ++t) acc[t] = 0.f;
-    if (e < a.E) {
-      const int r_end = (ks + 1) * P0_RS;
-#pragma unroll 4
-      for (int r = ks * P0_RS + rg; r < r_end; r += 18) {
-        const float w = __uint_as_float((uint32_t)__ldg(a.w_router + (size_t)r * a.E + e) << 16);
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t)
-          if (t < a.T)
-            acc[t] = fmaf(__uint_as_float((uint32_t)__ldg(a.x + (size_t)t * a.d + r) << 16), w,
-                          acc[t]);
-      }
+  const int th = threadIdx.x;
+  const int neb = (a.E + 63) / 64, nks = a.d / P0_RS;
+  float* red = scratch;                                   // [32][MAXT][64]
+  float* xr = scratch + 32 * MAXT * 64;                   // [MAXT][512]
+  for (int item = blockIdx.x; item < neb * nks; item += gridDim.x) {
+    const int eb = item % neb, ks = item / neb;
+    const int r0 = ks * P0_RS;
+    if (th < a.T * (P0_RS / 8)) {                         // one 16-byte chunk per thread
+      const int t = th / (P0_RS / 8), j = th % (P0_RS / 8);
+      const uint4 v = ld_nc_v4(a.x + (size_t)t * a.d + r0 + 8 * j);
+      float* dst = xr + t * P0_RS + 8 * j;
+      dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x); dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
+      dst[4] = bf16_lo(v.z); dst[5] = bf16_hi(v.z); dst[6] = bf16_lo(v.w); dst[7] = bf16_hi(v.w);
     }
-#pragma unroll
-    for (int t = 0; t < MAXT; ++t) red[(rg * MAXT + t) * P0_EC + el] = acc[t];
     __syncthreads();
-    if (th < a.T * P0_EC) {
-      const int t = th / P0_EC, l = th % P0_EC;
-      float s = 0.f;
-      for (int g = 0; g < 18; ++g) s += red[(g * MAXT + t) * P0_EC + l];
-      const int ee = ec * P0_EC + l;
-      if (ee < a.E) a.partial[((size_t)ks * a.T + t) * a.E + ee] = s;
+    if (th < 256) {
+      const int c = th & 7, rr = th >> 3;
+      const int e0 = eb * 64 + c * 8;
+      float acc[MAXT][8];
+#pragma unroll
+      for (int t = 0; t < MAXT; ++t)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[t][j] = 0.f;
+      if (e0 < a.E) {                                     // E % 8 == 0 on this path
+        uint4 w[P0_RS / 32];
+#pragma unroll
+        for (int i = 0; i < P0_RS / 32; ++i)
+          w[i] = ld_nc_v4(a.w_router + (size_t)(r0 + rr + 32 * i) * a.E + e0);
+#pragma unroll
+        for (int i = 0; i < P0_RS / 32; ++i) {
+          const float wv[8] = {bf16_lo(w[i].x), bf16_hi(w[i].x), bf16_lo(w[i].y), bf16_hi(w[i].y),
+                               bf16_lo(w[i].z), bf16_hi(w[i].z), bf16_lo(w[i].w), bf16_hi(w[i].w)};
+#pragma unroll
+          for (int t = 0; t < MAXT; ++t) {
+            if (t < a.T) {
+              const float xv = xr[t * P0_RS + rr + 32 * i];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) acc[t][j] = fmaf(xv, wv[j], acc[t][j]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < MAXT; ++t)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) red[(rr * MAXT + t) * 64 + c * 8 + j] = acc[t][j];
+    }
+    __syncthreads();
+    if (th < a.T * 64) {
+      const int t = th / 64, l = th % 64;
+      float sum = 0.f;
+      for (int g = 0; g < 32; ++g) sum += red[(g * MAXT + t) * 64 + l];
+      const int ee = eb * 64 + l;
+      if (ee < a.E) a.partial[((size_t)ks * a.T + t) * a.E + ee] = sum;
     }
     __syncthreads();
   }
@@ -198,11 +233,22 @@ __device__ void df_router_partials(const FusedArgs& a, float* red) {
 // x of all tokens -> fp16 in shared memory, features interleaved within
 // groups of 8 (0, 4, 1, 5, 2, 6, 3, 7) to match the weight fragments.
 __device__ bool df_load_x(const FusedArgs& a, uint16_t* xs) {
+  using namespace df;
   bool over = false;
   const int cpr = a.d / 8;
-  for (int c = threadIdx.x; c < a.T * cpr; c += blockDim.x) {
+  // every load of this thread first (at most XPT), then the conversions
+  uint4 vin[XPT];
+#pragma unroll
+  for (int i = 0; i < XPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c < a.T * cpr) vin[i] = ld_nc_v4(a.x + (size_t)c * 8);
+  }
+#pragma unroll
+  for (int i = 0; i < XPT; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c >= a.T * cpr) break;
     const int t = c / cpr, j = c % cpr;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + j);
+    const uint4 v = vin[i];
     float e[8];
     e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
     e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
@@ -233,10 +279,26 @@ struct Route {
   int* misc;         // [0] n_active, [1..32] scan scratch
 };
 
-__device__ void df_route(const FusedArgs& a, const Route& R) {
+__device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
   using namespace df;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nks = a.d / P0_RS, S = a.T * a.k;
+  // logits of every token: the K slices' partial sums in order, then the bias
+  // (each thread loads all partials of its logits before adding)
+  for (int i = threadIdx.x; i < a.T * a.E; i += blockDim.x) {
+    const int t = i / a.E, e = i % a.E;
+    float p[P0_MAXKS];
+#pragma unroll
+    for (int ks = 0; ks < P0_MAXKS; ++ks)
+      p[ks] = ks < nks ? __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e) : 0.f;
+    float acc = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < P0_MAXKS; ++ks)
+      if (ks < nks) acc += p[ks];
+    if (a.bias) acc += __ldg(a.bias + e);
+    logit_s[i] = acc;
+  }
+  __syncthreads();
   if (warp < a.T) {
     const int t = warp;
     float v[MAXE / 32];
@@ -245,14 +307,8 @@ __device__ void df_route(const FusedArgs& a, const Route& R) {
     for (int i = 0; i < MAXE / 32; ++i) {
       const int e = lane + 32 * i;
       v[i] = -INFINITY;
-      if (e < a.E) {
-        float acc = 0.f;
-        for (int ks = 0; ks < nks; ++ks) acc += __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e);
-        if (a.bias) acc += __ldg(a.bias + e);
-        v[i] = acc;
-      } else {
-        taken |= 1u << i;
-      }
+      if (e < a.E) v[i] = logit_s[t * a.E + e];
+      else taken |= 1u << i;
     }
     float my_v = 0.f, top = 0.f;
     int my_i = 0;
@@ -424,7 +480,10 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     moe_decode_fused_kernel(const __grid_constant__ CUtensorMap map_wg,
                             const __grid_constant__ CUtensorMap map_wu,
                             const __grid_constant__ CUtensorMap map_wd,
-                            const __grid_constant__ CUtensorMap map_h, const FusedArgs a) {
+                            const __grid_constant__ CUtensorMap map_h,
+                            const __grid_constant__ CUtensorMap map_sg,
+                            const __grid_constant__ CUtensorMap map_su,
+                            const __grid_constant__ CUtensorMap map_sd, const FusedArgs a) {
   using namespace df;
   constexpr int KB = G < 64 ? G : 64;      // K per block: one block lies in one scale group
   extern __shared__ uint8_t df_smem_raw[];
@@ -445,8 +504,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     R.w = reinterpret_cast<float*>(r + MAXS);
     R.counts = r + 2 * MAXS;
     R.active = R.counts + MAXE;
-    R.pos = R.active + MAXE;
-    R.offsets = R.pos + MAXE;
+    R.pos = reinterpret_cast<int32_t*>(ring) + MAXT * MAXE;   // after the P1 logits
+    R.offsets = R.active + MAXE;
     R.rowtok = R.offsets + MAXE + 1;
     R.slotrow = R.rowtok + MAXS;
     R.misc = R.slotrow + MAXS;
@@ -468,6 +527,9 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     prefetch_tmap(&map_wu);
     prefetch_tmap(&map_wd);
     prefetch_tmap(&map_h);
+    prefetch_tmap(&map_sg);
+    prefetch_tmap(&map_su);
+    prefetch_tmap(&map_sd);
   }
   // ---- P0: x in fp16 (this CTA's copy), router partials (shared work)
   if (df_load_x(a, xs)) atomicOr(a.err, kErrRange);
@@ -475,7 +537,9 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   df_router_partials(a, reinterpret_cast<float*>(ring));
   bool ok = df_sync_grid(a.sync, 0, a.err, flag, abort_flag);
   // ---- P1: routes and grouping, in every CTA
-  if (ok) df_route(a, R);
+  if (ok) df_route(a, R, reinterpret_cast<float*>(ring));
+  // the ring held generic-proxy data (P0, P1); the TMA writes into it next
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   const int n_active = ok ? R.misc[0] : 0;
   const int S = a.T * a.k;
 
@@ -497,25 +561,27 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             break;
           }
           uint8_t* sl = ring + s * SLOT;
-          mbar_arrive_expect_tx(&full[s], 2 * P2_ROWS * (P2_KST / 2));
+          constexpr int SG = P2_ROWS * (P2_KST / G) * 2;   // scale bytes per matrix
+          mbar_arrive_expect_tx(&full[s], 2 * P2_ROWS * (P2_KST / 2) + 2 * SG);
 #pragma unroll
           for (int b = 0; b < P2_KST / 256; ++b) {
             tma_load_2d(sl + b * 2048, &map_wg, kc * (P2_KST / 2) + b * 128, wrow, &full[s]);
             tma_load_2d(sl + 8192 + b * 2048, &map_wu, kc * (P2_KST / 2) + b * 128, wrow,
                         &full[s]);
           }
+          tma_load_2d(sl + P2_SC, &map_sg, kc * (P2_KST / G), wrow, &full[s]);
+          tma_load_2d(sl + P2_SC + SG, &map_su, kc * (P2_KST / G), wrow, &full[s]);
         }
       }
     }
   } else {
     const int ks = warp;                    // this warp's 128 K of each stage
-    const int NG = a.d / G;                 // groups per weight row
+    constexpr int SGR = P2_KST / G;         // scale groups per row in a stage
     for (int u = blockIdx.x; u < units2; u += gridDim.x) {
       const int e = R.active[u / FB2], fb = u % FB2;
       const int cnt = R.counts[e], prow = R.offsets[e];
       const int tok = R.rowtok[prow + min(g8, cnt - 1)];
       const uint16_t* xr = xs + (size_t)tok * XP;
-      const size_t srow = (size_t)(e * a.n + fb * P2_ROWS + g8) * NG;
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       bool failed = false;
       for (int kc = 0; kc < KS2; ++kc, ++g) {
@@ -531,7 +597,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           const int kb = k0 + bi * KB;
           uint32_t b[KB / 8];
           df_bfrag<KB>(xr + kb + t * (KB / 4), b);
-          const int grp = kb / G;
+          const int grp = (ks * 128 + bi * KB) / G;       // scale group within the stage
           const int o = (ks & 1) * 64 + (bi * KB + t * (KB / 4)) / 2;   // byte in the box row
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
@@ -540,9 +606,10 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             df_words<KB>(tile, g8, o, w0, w8);
             float c[4];
             df_block<KB>(w0, w8, b, c);
-            const uint16_t* sp = (m == 0 ? a.s_gate : a.s_up) + srow + grp;
-            const float s0 = __half2float(__ushort_as_half(__ldg(sp)));
-            const float s8 = __half2float(__ushort_as_half(__ldg(sp + 8 * NG)));
+            const uint16_t* sp = reinterpret_cast<const uint16_t*>(sl + P2_SC) +
+                                 m * P2_ROWS * SGR + g8 * SGR + grp;
+            const float s0 = df_half(sp);
+            const float s8 = df_half(sp + 8 * SGR);
             acc[m][0] = fmaf(s0, c[0], acc[m][0]);
             acc[m][1] = fmaf(s0, c[1], acc[m][1]);
             acc[m][2] = fmaf(s8, c[2], acc[m][2]);
@@ -594,20 +661,21 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             break;
           }
           uint8_t* sl = ring + s * SLOT;
-          mbar_arrive_expect_tx(&full[s], P3_ROWS * (P3_KST / 2) + MAXT * P3_KST * 2);
+          mbar_arrive_expect_tx(&full[s], P3_ROWS * (P3_KST / 2) + MAXT * P3_KST * 2 +
+                                              P3_ROWS * (a.n / G) * 2);
           tma_load_2d(sl, &map_wd, kc * (P3_KST / 2), wrow, &full[s]);
-          tma_load_2d(sl + 8192, &map_h, kc * P3_KST, prow, &full[s]);
+          tma_load_2d(sl + P3_H, &map_h, kc * P3_KST, prow, &full[s]);
+          tma_load_2d(sl + P3_SC, &map_sd, 0, wrow, &full[s]);     // the unit's scale rows
         }
       }
     }
   } else {
     const int rg = warp & 3, kh = warp >> 2;
-    const int NG = a.n / G;
+    const int NG = a.n / G;                 // scale groups per down row
     for (int u = blockIdx.x; u < units3; u += gridDim.x) {
       const int e = R.active[u / FB3], fb = u % FB3;
       const int cnt = R.counts[e], prow = R.offsets[e];
       const int hrow = g8 < cnt ? g8 : 0;
-      const size_t srow = (size_t)(e * a.d + fb * P3_ROWS + rg * 16 + g8) * NG;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       bool failed = false;
       for (int kc = 0; kc < KS3; ++kc, ++g) {
@@ -617,7 +685,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           break;
         }
         const uint8_t* sl = ring + s * SLOT;
-        const uint16_t* hr = reinterpret_cast<const uint16_t*>(sl + 8192) + hrow * P3_KST;
+        const uint16_t* hr = reinterpret_cast<const uint16_t*>(sl + P3_H) + hrow * P3_KST;
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(sl + P3_SC) + (rg * 16 + g8) * NG;
         const uint8_t* tile = sl + rg * 16 * 128;
 #pragma unroll
         for (int bi = 0; bi < 128 / KB; ++bi) {
@@ -629,8 +698,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           float c[4];
           df_block<KB>(w0, w8, b, c);
           const int grp = (kc * P3_KST + kl) / G;
-          const float s0 = __half2float(__ushort_as_half(__ldg(a.s_down + srow + grp)));
-          const float s8 = __half2float(__ushort_as_half(__ldg(a.s_down + srow + 8 * NG + grp)));
+          const float s0 = df_half(sc + grp);
+          const float s8 = df_half(sc + 8 * NG + grp);
           acc[0] = fmaf(s0, c[0], acc[0]);
           acc[1] = fmaf(s0, c[1], acc[1]);
           acc[2] = fmaf(s8, c[2], acc[2]);
@@ -690,7 +759,12 @@ bool decode_fused_fits(int T, int d, int E, int k, int n, int G) {
   using namespace df;
   if (T < 1 || T > MAXT || k > MAXK || E > MAXE) return false;
   if (G != 32 && G != 64 && G != 128) return false;
-  if (d % P2_KST || d % P0_RS || n % P3_KST || n % P2_ROWS || d % P3_ROWS) return false;
+  if (d % P2_KST || d % P0_RS || d / P0_RS > P0_MAXKS || n % P3_KST || n % P2_ROWS ||
+      d % P3_ROWS || E % 8 || T * d > 8 * XPT * THREADS)
+    return false;
+  // scale tiles by TMA: rows of at least 16 bytes, at most 256 groups, fitting the stage
+  if ((P2_KST / G) % 8 || (n / G) % 8 || n / G > 256 || P3_SC + P3_ROWS * (n / G) * 2 > SLOT)
+    return false;
   return Smem::of(T, d).total + 1024 <= 113 * 1024;
 }
 
@@ -722,7 +796,8 @@ static cudaError_t launch_fused_g(const CUtensorMap* maps, const FusedArgs& a, i
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], a);
+  return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                            maps[6], a);
 }
 
 cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, const float* bias,
@@ -760,7 +835,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, con
   a.k = k;
   a.n = n;
   a.G = G;
-  CUtensorMap maps[4];
+  CUtensorMap maps[7];
   if (encode_tmap_2d(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, q_gate, d / 2, (uint64_t)E * n, d / 2,
                      128, P2_ROWS, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS ||
@@ -772,6 +847,17 @@ cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, con
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS ||
       encode_tmap_2d(&maps[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.h, n, S, (uint64_t)n * 2, P3_KST,
                      MAXT, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS ||
+      // scales: gate/up 1024 / G groups x 16 rows per stage, down n / G groups
+      // x 64 rows (a unit's whole scale rows) per stage
+      encode_tmap_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s_gate, d / G, (uint64_t)E * n,
+                     (uint64_t)(d / G) * 2, P2_KST / G, P2_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS ||
+      encode_tmap_2d(&maps[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s_up, d / G, (uint64_t)E * n,
+                     (uint64_t)(d / G) * 2, P2_KST / G, P2_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS ||
+      encode_tmap_2d(&maps[6], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, s_down, n / G, (uint64_t)E * d,
+                     (uint64_t)(n / G) * 2, n / G, P3_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(a.sync, 0, 16, s);
