@@ -285,18 +285,29 @@ __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
   const int nks = a.d / P0_RS, S = a.T * a.k;
   // logits of every token: the K slices' partial sums in order, then the bias
   // (each thread loads all partials of its logits before adding)
-  for (int i = threadIdx.x; i < a.T * a.E; i += blockDim.x) {
-    const int t = i / a.E, e = i % a.E;
-    float p[P0_MAXKS];
+  // (four logits per thread per pass: 32 loads in flight)
+  for (int i0 = threadIdx.x; i0 < a.T * a.E; i0 += 4 * blockDim.x) {
+    float p[4][P0_MAXKS];
 #pragma unroll
-    for (int ks = 0; ks < P0_MAXKS; ++ks)
-      p[ks] = ks < nks ? __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e) : 0.f;
-    float acc = 0.f;
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int t = i / a.E, e = i % a.E;
 #pragma unroll
-    for (int ks = 0; ks < P0_MAXKS; ++ks)
-      if (ks < nks) acc += p[ks];
-    if (a.bias) acc += __ldg(a.bias + e);
-    logit_s[i] = acc;
+      for (int ks = 0; ks < P0_MAXKS; ++ks)
+        p[u][ks] = (i < a.T * a.E && ks < nks)
+                       ? __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i >= a.T * a.E) break;
+      float acc = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < P0_MAXKS; ++ks)
+        if (ks < nks) acc += p[u][ks];
+      if (a.bias) acc += __ldg(a.bias + i % a.E);
+      logit_s[i] = acc;
+    }
   }
   __syncthreads();
   if (warp < a.T) {

@@ -57,7 +57,6 @@ constexpr int BM = 128;                    // weight rows per slot (TMEM lanes)
 constexpr int NT = kTileRows;              // token rows per unit (max MMA N)
 constexpr int BK = 64;                     // K per stage
 constexpr int RAW_ST = 8;                  // packed-weight ring depth
-constexpr int B_ST = 4;                    // token-row ring depth
 constexpr int A_ST = 4;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
@@ -76,14 +75,21 @@ struct Roles {
   static constexpr int THREADS = (W_EPI + 4) * 32;
 };
 
-constexpr int RAW_OFF = 0;                                        // [RAW_ST][2][RAW_BYTES]
-constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;           // [B_ST][B_BYTES]
-constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;                   // [2 * BM][STG_PITCH] fp16
-constexpr int STG_BYTES = 2 * BM * STG_PITCH * 2;
-constexpr int BAR_OFF = STG_OFF + STG_BYTES;
-constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
-constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-constexpr int SMEM = 1024 + MISC_OFF + 64;
+// Shared memory per operation: gate/up writes one 128-feature slice per unit
+// (SwiGLU merges the two slots), so its staging tile is half the size of
+// down's and the space goes to two more token-row stages.
+template <int OP>
+struct Lay {
+  static constexpr int B_ST = OP == 0 ? 6 : 4;                      // token-row ring depth
+  static constexpr int RAW_OFF = 0;                                 // [RAW_ST][2][RAW_BYTES]
+  static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;    // [B_ST][B_BYTES]
+  static constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;            // [slices * BM][STG_PITCH]
+  static constexpr int STG_BYTES = (OP == 0 ? 1 : 2) * BM * STG_PITCH * 2;
+  static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
+  static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM = 1024 + MISC_OFF + 64;
+};
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t A_COL = 256;
@@ -228,13 +234,15 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
                           const __grid_constant__ CUtensorMap map_q1,
                           const __grid_constant__ CUtensorMap map_b, const TcArgs args) {
   using namespace tc;
+  using Ly = Lay<OP>;
+  constexpr int B_ST = Ly::B_ST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sRaw = smem + RAW_OFF;
-  uint8_t* sB = smem + B_OFF;
-  uint16_t* sStg = reinterpret_cast<uint16_t*>(smem + STG_OFF);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint8_t* sRaw = smem + Ly::RAW_OFF;
+  uint8_t* sB = smem + Ly::B_OFF;
+  uint16_t* sStg = reinterpret_cast<uint16_t*>(smem + Ly::STG_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFF);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + RAW_ST;
   uint64_t* b_full = raw_empty + RAW_ST;
@@ -243,8 +251,8 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   uint64_t* a_empty = a_full + A_ST;
   uint64_t* acc_full = a_empty + A_ST;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFF + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -494,16 +502,14 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * sw);
         raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * (sw ^ 1));
       }
-      if (g >= A_ST && !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
-        break;
-      __syncwarp();       // converged before the .sync.aligned TMEM stores
-      tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
+      // gate/up: both slots are dequantised into registers before this warp
+      // waits for its A stage, so a stage the MMAs release is refilled at
+      // once; down (three warpgroups at 96 registers) has no room for that
+      // and dequantises slot by slot after the wait.
+      auto dq_slot = [&](int m, uint32_t(&out)[32]) {
         const uint32_t sc_a = sc2[m][0], sc_b = sc2[m][1];
         const uint32_t words[8] = {raw[m][0].x, raw[m][0].y, raw[m][0].z, raw[m][0].w,
                                    raw[m][1].x, raw[m][1].y, raw[m][1].z, raw[m][1].w};
-        uint32_t out[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           // gate/up: the grouped copy of x is interleaved; down: h is
@@ -511,12 +517,35 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
           if (OP == 0 || ILV) dequant8_interleaved(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
           else dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
         }
-        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
+      };
+      if constexpr (OP == 0) {
+        uint32_t out0[32], out1[32];
+        dq_slot(0, out0);
+        dq_slot(1, out1);
+        // The packed words have been consumed, so the next TMA write into
+        // this raw stage cannot overtake a shared-memory load still in flight.
+        mbar_arrive(&raw_empty[sr]);
+        if (g >= A_ST &&
+            !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
+          break;
+        __syncwarp();       // converged before the .sync.aligned TMEM stores
+        tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
+        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64, out0);
+        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + 32, out1);
+      } else {
+        if (g >= A_ST &&
+            !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
+          break;
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          uint32_t out[32];
+          dq_slot(m, out);
+          tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
+        }
+        mbar_arrive(&raw_empty[sr]);   // the packed words have been consumed
       }
-      // The packed words have been consumed (the dequantisation above used
-      // them), so the next TMA write into this raw stage cannot overtake a
-      // shared-memory load still in flight.
-      mbar_arrive(&raw_empty[sr]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&a_full[sa]);
@@ -647,7 +676,8 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
     return cudaErrorInvalidValue;
   {
     cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP, ILV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::Lay<OP>::SMEM);
     if (e != cudaSuccess) return e;
   }
   const int num_sms = sm_count();
@@ -677,7 +707,8 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::Roles<OP>::THREADS, tc::SMEM, s>>>(m0, m1, mb, a);
+  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP>::SMEM, s>>>(m0, m1,
+                                                                                        mb, a);
   return cudaGetLastError();
 }
 
