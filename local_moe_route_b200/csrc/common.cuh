@@ -185,6 +185,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+// Before a thread releases a shared-memory slot that TMA (the async proxy)
+// will overwrite: orders this thread's earlier generic reads of the slot
+// before those writes.  Without it a load whose result is consumed only
+// later (the compiler may schedule that arithmetic after the release) can
+// still be in flight when the next copy lands.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

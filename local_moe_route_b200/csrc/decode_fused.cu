@@ -627,6 +627,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             acc[m][3] = fmaf(s8, c[3], acc[m][3]);
           }
         }
+        fence_proxy_async_smem();           // this stage's loads before its next TMA write
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
@@ -716,6 +717,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           acc[2] = fmaf(s8, c[2], acc[2]);
           acc[3] = fmaf(s8, c[3], acc[3]);
         }
+        fence_proxy_async_smem();           // this stage's loads before its next TMA write
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }

@@ -301,7 +301,8 @@ __global__ void __launch_bounds__(dk::THREADS, NMAT == 1 ? 3 : 2)
             }
           }
         }
-        // the stage's words were consumed by the MMAs above; release it
+        // release the stage; the fence orders its loads before the next TMA write
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }

@@ -522,8 +522,9 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         uint32_t out0[32], out1[32];
         dq_slot(0, out0);
         dq_slot(1, out1);
-        // The packed words have been consumed, so the next TMA write into
-        // this raw stage cannot overtake a shared-memory load still in flight.
+        // Release the raw stage: the fence orders the loads of its words
+        // before the next TMA write into it.
+        fence_proxy_async_smem();
         mbar_arrive(&raw_empty[sr]);
         if (g >= A_ST &&
             !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
@@ -544,7 +545,8 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
           dq_slot(m, out);
           tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
         }
-        mbar_arrive(&raw_empty[sr]);   // the packed words have been consumed
+        fence_proxy_async_smem();      // the words' loads before the next TMA write
+        mbar_arrive(&raw_empty[sr]);
       }
       tmem_st_wait();
       tc_fence_before();
