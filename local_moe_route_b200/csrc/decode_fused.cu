@@ -310,27 +310,33 @@ __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
     }
   }
   __syncthreads();
-  if (warp < a.T) {
-    const int t = warp;
-    float v[MAXE / 32];
+  // top k of each token by two warps: warp 2t + hf selects the k best of its
+  // half of the experts (exact ties to the lower index, NaN never wins), then
+  // warp 2t merges the two lists of k with the same order.  Any of the
+  // token's k best lies among its half's k best, so the merge is exact.
+  float* cand_v = logit_s + MAXT * MAXE;                  // [MAXT][2][MAXK]
+  int* cand_i = reinterpret_cast<int*>(cand_v + MAXT * 2 * MAXK);
+  const int half = (a.E + 1) / 2;
+  if (warp < 2 * a.T) {
+    const int t = warp >> 1, hf = warp & 1;
+    const int lo = hf * half, hi = min(a.E, lo + half);
+    float v[MAXE / 64];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < MAXE / 32; ++i) {
-      const int e = lane + 32 * i;
+    for (int i = 0; i < MAXE / 64; ++i) {
+      const int e = lo + lane + 32 * i;
       v[i] = -INFINITY;
-      if (e < a.E) v[i] = logit_s[t * a.E + e];
+      if (e < hi) v[i] = logit_s[t * a.E + e];
       else taken |= 1u << i;
     }
-    float my_v = 0.f, top = 0.f;
-    int my_i = 0;
     for (int j = 0; j < a.k; ++j) {
       float best = -INFINITY;
       int bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < MAXE / 32; ++i) {
+      for (int i = 0; i < MAXE / 64; ++i) {
         if (!((taken >> i) & 1u)) {
-          const float c = (v[i] != v[i]) ? -INFINITY : v[i];   // NaN never wins
-          const int e = lane + 32 * i;
+          const float c = (v[i] != v[i]) ? -INFINITY : v[i];
+          const int e = lo + lane + 32 * i;
           if (c > best || (c == best && e < bi)) {
             best = c;
             bi = e;
@@ -346,7 +352,57 @@ __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
           bi = oi;
         }
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (bi != 0x7fffffff && ((bi - lo) & 31) == lane) taken |= 1u << ((bi - lo) >> 5);
+      if (lane == 0) {
+        cand_v[(t * 2 + hf) * MAXK + j] = best;
+        cand_i[(t * 2 + hf) * MAXK + j] = bi;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp < a.T) {
+    const int t = warp;
+    // the 2k candidates, lane l holding numbers l and l + 32 (candidate c is
+    // number c of the first half's list for c < k, else c - k of the second)
+    float cv[2];
+    int ci[2];
+    bool taken[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = lane + 32 * u;
+      cv[u] = -INFINITY;
+      ci[u] = 0x7fffffff;
+      if (c < 2 * a.k) {
+        const int hf = c < a.k ? 0 : 1, j = c < a.k ? c : c - a.k;
+        cv[u] = cand_v[(t * 2 + hf) * MAXK + j];
+        ci[u] = cand_i[(t * 2 + hf) * MAXK + j];
+      }
+      taken[u] = ci[u] == 0x7fffffff;
+    }
+    float my_v = 0.f, top = 0.f;
+    int my_i = 0;
+    for (int j = 0; j < a.k; ++j) {
+      float best = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!taken[u] && (cv[u] > best || (cv[u] == best && ci[u] < bi))) {
+          best = cv[u];
+          bi = ci[u];
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ob > best || (ob == best && oi < bi)) {
+          best = ob;
+          bi = oi;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (!taken[u] && ci[u] == bi) taken[u] = true;
       if (j == 0) top = best;
       if (lane == j) {
         my_v = best;
@@ -515,7 +571,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     R.w = reinterpret_cast<float*>(r + MAXS);
     R.counts = r + 2 * MAXS;
     R.active = R.counts + MAXE;
-    R.pos = reinterpret_cast<int32_t*>(ring) + MAXT * MAXE;   // after the P1 logits
+    // after the P1 logits and the top-k candidates
+    R.pos = reinterpret_cast<int32_t*>(ring) + MAXT * MAXE + 2 * MAXT * 2 * MAXK;
     R.offsets = R.active + MAXE;
     R.rowtok = R.offsets + MAXE + 1;
     R.slotrow = R.rowtok + MAXS;

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(rs::THREADS)
   const int k_begin = split * rows_per_split;
   const int k_end = min(d, k_begin + rows_per_split);
   const bool even_e = (E & 1) == 0;
-  for (int t0 = 0; t0 < T; t0 += TT) {
+  for (int t0 = blockIdx.z * TT; t0 < T; t0 += gridDim.z * TT) {
     float acc[TT][2];
 #pragma unroll
     for (int j = 0; j < TT; ++j) acc[j][0] = acc[j][1] = 0.f;
@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_router_logits_simt(const uint16_t* x, const uint16_t* w_router, int T, int d,
                                       int E, int ksplit, float* partial, cudaStream_t s) {
   const int rows = (d + ksplit - 1) / ksplit;
-  dim3 grid((E + rs::EXPERTS - 1) / rs::EXPERTS, ksplit);
+  // token tiles spread over grid.z (each block loops if there are more)
+  const int tiles = (T + rs::TT - 1) / rs::TT;
+  dim3 grid((E + rs::EXPERTS - 1) / rs::EXPERTS, ksplit, tiles < 65535 ? tiles : 65535);
   router_logits_simt_kernel<<<grid, rs::THREADS, 0, s>>>(x, w_router, T, d, E, rows, partial);
   if (ksplit > 1) {
     dim3 rgrid((E + 31) / 32, T);

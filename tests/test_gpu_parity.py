@@ -308,6 +308,49 @@ def test_forward_edge_cases(dims, dev):
     _check_forward(L, y, ids, np.arange(dims["T"]), dims["k"], dims["group"], str(dims))
 
 
+# Batches of at most four tokens with d % 1024 == 0 run as one persistent
+# launch (router partials, top-k in two warps per token and merge, grouping,
+# both projections, combine); these shapes reach its corners.
+FUSED_EDGE = [
+    dict(T=1, d=1024, E=8, k=8, n=256, group=32),        # k = E: a half has fewer than k
+    dict(T=3, d=1024, E=64, k=32, n=512, group=64),      # k = 32: 64 candidates to merge
+    dict(T=4, d=2048, E=1024, k=4, n=1024, group=128),   # E = 1024, group 128
+    dict(T=2, d=1024, E=24, k=5, n=512, group=64),       # E not a power of two
+]
+
+
+@pytest.mark.parametrize("dims", FUSED_EDGE,
+                         ids=lambda d: "T{T}_d{d}_E{E}_k{k}_n{n}_g{group}".format(**d))
+def test_fused_decode_edge_cases(dims, dev):
+    import bench
+    assert bench.fused_decode(dims["T"], dims["d"], dims["E"], dims["k"], dims["n"],
+                              dims["group"])
+    L = Layer.custom(dev, seed=45 + dims["E"], **dims)
+    y, ids, w = L.forward()
+    assert_device_ok()
+    _check_forward(L, y, ids, np.arange(dims["T"]), dims["k"], dims["group"], "fused " + str(dims))
+
+
+def test_fused_decode_exact_ties_go_to_the_lower_index(dev):
+    """Integer-valued x and W_r (times 2^-4) make the logits exact in fp32 and
+    full of exact ties; the fused kernel's top-k must match the oracle's,
+    lowest index first, bit for bit."""
+    T, d, E, k = 4, 1024, 64, 8
+    L = Layer.custom(dev, T=T, d=d, E=E, k=k, n=512, group=64, seed=61)
+    rng = np.random.default_rng(9)
+    L.inp["x"] = bf16_bits(rng.integers(-2, 3, (T, d)).astype(np.float32))
+    L.inp["w_router"] = bf16_bits(rng.integers(-1, 2, (d, E)).astype(np.float32) / 16)
+    L.x = torch.from_numpy(L.inp["x"]).to(dev).view(torch.bfloat16)
+    L.w_router = torch.from_numpy(L.inp["w_router"]).to(dev).view(torch.bfloat16)
+    y, ids, w = L.forward()
+    assert_device_ok()
+    lg_ref, ids_ref, w_ref = oracle_routes(L)
+    srt = -np.sort(-lg_ref, axis=1)[:, :k + 1]
+    assert np.any(np.diff(srt, axis=1) == 0), "the case should contain exact ties"
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.max(np.abs(w.cpu().numpy() - w_ref)) <= 1e-6
+
+
 def test_forward_all_tokens_one_expert(dev):
     """A bias that sends every token to the same two experts: 300 rows per
     expert (three row tiles of the tensor-core kernel), the rest empty."""
