@@ -13,6 +13,8 @@
 //   P0  router partial logits (items of 512 rows of W_r x 64 experts);
 //       every CTA also converts x of all tokens to fp16 in shared memory;
 //   --- grid barrier
+//   P0b the logits, each summed once from the partials (spread over CTAs);
+//   --- grid barrier
 //   P1  every CTA sums the partials, picks each token's top k (exact ties to
 //       the lower expert index), the softmax weights, and groups the T*k
 //       slots by expert (counts, offsets, stable order) in its own shared
@@ -52,6 +54,7 @@ constexpr int ST = 3;                     // ring stages
 constexpr int SLOT = 18432;               // bytes per ring stage
 constexpr int P2_SC = 16384;              // offset of the gate/up scales in a stage
 constexpr int P3_H = 8192, P3_SC = 10240; // offsets of h and of the down scales
+constexpr int PF = 6;                     // stages the producer prefetches into L2 ahead
 constexpr int P2_ROWS = 16;               // gate/up unit: 16 rows, K split 8 ways
 constexpr int P2_KST = 1024;              // gate/up K per stage
 constexpr int P3_ROWS = 64;               // down unit: 4 row groups x 2 K halves
@@ -94,6 +97,7 @@ struct FusedArgs {
   int32_t* ids_out;          // [T][k] or null
   float* w_out;              // [T][k] or null
   float* partial;            // [d / 512][T][E]
+  float* logits;             // [T][E]
   uint16_t* h;               // [T*k][n] fp16, features interleaved within 8
   float* rows;               // [T*k][d] fp32
   unsigned* sync;            // [4] zeroed before the launch
@@ -279,36 +283,34 @@ struct Route {
   int* misc;         // [0] n_active, [1..32] scan scratch
 };
 
+// P0b: the logits, each once: the K slices' partial sums in order, then the
+// bias.  Spread over the CTAs (every CTA reading all partials would make 64
+// KB of L2 the hot spot of every SM at once).
+__device__ void df_logits(const FusedArgs& a) {
+  using namespace df;
+  const int nks = a.d / P0_RS;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.T * a.E;
+       i += gridDim.x * blockDim.x) {
+    const int t = i / a.E, e = i % a.E;
+    float p[P0_MAXKS];
+#pragma unroll
+    for (int ks = 0; ks < P0_MAXKS; ++ks)
+      p[ks] = ks < nks ? __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e) : 0.f;
+    float acc = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < P0_MAXKS; ++ks)
+      if (ks < nks) acc += p[ks];
+    if (a.bias) acc += __ldg(a.bias + e);
+    a.logits[i] = acc;
+  }
+}
+
 __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
   using namespace df;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nks = a.d / P0_RS, S = a.T * a.k;
-  // logits of every token: the K slices' partial sums in order, then the bias
-  // (each thread loads all partials of its logits before adding)
-  // (four logits per thread per pass: 32 loads in flight)
-  for (int i0 = threadIdx.x; i0 < a.T * a.E; i0 += 4 * blockDim.x) {
-    float p[4][P0_MAXKS];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * blockDim.x;
-      const int t = i / a.E, e = i % a.E;
-#pragma unroll
-      for (int ks = 0; ks < P0_MAXKS; ++ks)
-        p[u][ks] = (i < a.T * a.E && ks < nks)
-                       ? __ldcg(a.partial + ((size_t)ks * a.T + t) * a.E + e) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * blockDim.x;
-      if (i >= a.T * a.E) break;
-      float acc = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < P0_MAXKS; ++ks)
-        if (ks < nks) acc += p[u][ks];
-      if (a.bias) acc += __ldg(a.bias + i % a.E);
-      logit_s[i] = acc;
-    }
-  }
+  // logits of every token (summed once, by all CTAs together, in P0b)
+  for (int i = threadIdx.x; i < a.T * a.E; i += blockDim.x) logit_s[i] = __ldcg(a.logits + i);
   __syncthreads();
   // top k of each token by two warps: warp 2t + hf selects the k best of its
   // half of the experts (exact ties to the lower index, NaN never wins), then
@@ -604,6 +606,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   __syncthreads();
   df_router_partials(a, reinterpret_cast<float*>(ring));
   bool ok = df_sync_grid(a.sync, 0, a.err, flag, abort_flag);
+  if (ok) df_logits(a);
+  ok = df_sync_grid(a.sync, 1, a.err, flag, abort_flag) && ok;
   // ---- P1: routes and grouping, in every CTA
   if (ok) df_route(a, R, reinterpret_cast<float*>(ring));
   // the ring held generic-proxy data (P0, P1); the TMA writes into it next
@@ -618,10 +622,27 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   if (warp == CONS) {
     if (lane == 0) {
       bool stop = false;
+      // stage q of this CTA's gate/up stream: unit blockIdx.x + (q / KS2) * gridDim.x, K block q % KS2
+      auto prefetch2 = [&](int q) {
+        const int u = blockIdx.x + (q / KS2) * (int)gridDim.x;
+        if (u >= units2) return;
+        const int kc = q % KS2;
+        const int wrow = R.active[u / FB2] * a.n + (u % FB2) * P2_ROWS;
+#pragma unroll
+        for (int b = 0; b < P2_KST / 256; ++b) {
+          tma_prefetch_2d(&map_wg, kc * (P2_KST / 2) + b * 128, wrow);
+          tma_prefetch_2d(&map_wu, kc * (P2_KST / 2) + b * 128, wrow);
+        }
+        tma_prefetch_2d(&map_sg, kc * (P2_KST / G), wrow);
+        tma_prefetch_2d(&map_su, kc * (P2_KST / G), wrow);
+      };
+      for (int q = 0; q < PF; ++q) prefetch2(q);
+      int q2 = 0;
       for (int u = blockIdx.x; u < units2 && !stop; u += gridDim.x) {
         const int e = R.active[u / FB2];
         const int wrow = e * a.n + (u % FB2) * P2_ROWS;
-        for (int kc = 0; kc < KS2; ++kc, ++g) {
+        for (int kc = 0; kc < KS2; ++kc, ++g, ++q2) {
+          prefetch2(q2 + PF);
           const int s = g % ST;
           if (g >= (uint32_t)ST &&
               !mbar_wait(&empty[s], ((g / ST) - 1) & 1, abort_flag, a.err)) {
@@ -710,7 +731,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       named_barrier_sync(1, CONS * 32);     // red is reused by the next unit
     }
   }
-  ok = df_sync_grid(a.sync, 1, a.err, flag, abort_flag) && ok;
+  ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
 
   // ---- P3: down, units (expert, 64 rows): 4 row groups x 2 K halves
   const int FB3 = a.d / P3_ROWS, KS3 = a.n / P3_KST;
@@ -718,11 +739,23 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   if (warp == CONS) {
     if (lane == 0) {
       bool stop = false;
+      auto prefetch3 = [&](int q) {
+        const int u = blockIdx.x + (q / KS3) * (int)gridDim.x;
+        if (u >= units3) return;
+        const int kc = q % KS3;
+        const int e = R.active[u / FB3];
+        const int wrow = e * a.d + (u % FB3) * P3_ROWS;
+        tma_prefetch_2d(&map_wd, kc * (P3_KST / 2), wrow);
+        if (kc == 0) tma_prefetch_2d(&map_sd, 0, wrow);
+      };
+      for (int q = 0; q < PF; ++q) prefetch3(q);
+      int q3 = 0;
       for (int u = blockIdx.x; u < units3 && !stop; u += gridDim.x) {
         const int e = R.active[u / FB3];
         const int wrow = e * a.d + (u % FB3) * P3_ROWS;
         const int prow = R.offsets[e];
-        for (int kc = 0; kc < KS3; ++kc, ++g) {
+        for (int kc = 0; kc < KS3; ++kc, ++g, ++q3) {
+          prefetch3(q3 + PF);
           const int s = g % ST;
           if (g >= (uint32_t)ST &&
               !mbar_wait(&empty[s], ((g / ST) - 1) & 1, abort_flag, a.err)) {
@@ -795,7 +828,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       named_barrier_sync(1, CONS * 32);
     }
   }
-  ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
+  ok = df_sync_grid(a.sync, 3, a.err, flag, abort_flag) && ok;
 
   // ---- P4: combine, fp32 in slot order j = 0 .. k-1, one rounding to bf16
   if (ok) {
@@ -842,7 +875,8 @@ size_t decode_fused_scratch(int T, int d, int E, int k, int n) {
   // partial logits, h, rows, sync words (each region 256-byte aligned)
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t S = (size_t)T * k;
-  return up((size_t)(d / df::P0_RS) * T * E * 4) + up(S * n * 2) + up(S * d * 4) + 256;
+  return up((size_t)(d / df::P0_RS) * T * E * 4) + up((size_t)T * E * 4) + up(S * n * 2) +
+         up(S * d * 4) + 256;
 }
 
 template <int G>
@@ -893,6 +927,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, con
   a.w_out = w_out;
   a.partial = reinterpret_cast<float*>(base);
   base += up((size_t)(d / P0_RS) * T * E * 4);
+  a.logits = reinterpret_cast<float*>(base);
+  base += up((size_t)T * E * 4);
   a.h = reinterpret_cast<uint16_t*>(base);
   base += up(S * n * 2);
   a.rows = reinterpret_cast<float*>(base);

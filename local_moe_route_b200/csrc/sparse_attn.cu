@@ -12,12 +12,12 @@
 // Small query batches (decode, speculative verify) are bound by the bytes of
 // the selected rows, 2 * Hkv * D * 2 bytes per position per query.  Two
 // kernels, split-K style:
-//   1. one CTA per (query, KV head, slice of 128 index slots): every thread
-//      takes one slot, reads its K row (16-byte loads) and forms the scores of
-//      the G query heads that share the KV head; the slice's softmax maximum
-//      and sum per head go to shared memory; then thread d accumulates
-//      sum_p exp(s - m) V[p][d] over the slice (V rows read whole by the
-//      block, 256 bytes per row), fp32;
+//   1. one CTA per (query, KV head, slice of 128 index slots): the slice's
+//      selected K and V rows are copied into shared memory (cp.async, all
+//      issued before one wait); every thread takes one slot and forms the
+//      scores of the G query heads that share the KV head; the slice's
+//      softmax maximum and sum per head stay in shared memory; thread d
+//      accumulates sum_p exp(s - m) V[p][d] over the slice, fp32;
 //   2. one CTA per (query, head) rescales and adds the slices' partial sums
 //      (max-subtracted exponentials, fixed order) and rounds to bf16.
 #include "common.cuh"
@@ -39,17 +39,18 @@ __global__ void __launch_bounds__(sa::THREADS)
                              float* __restrict__ part_o, float* __restrict__ part_ml,
                              unsigned* err) {
   using namespace sa;
+  constexpr int RP = D + 8;                  // halves per staged row (16 bytes of padding)
   const int split = blockIdx.x, hk = blockIdx.y, t = blockIdx.z;
   const int G = Hq / Hkv;
-  __shared__ float qs[MAXG][D];
-  __shared__ float ws[MAXG][SLICE];          // scores, then exp(s - m)
-  __shared__ int rows[SLICE];
-  __shared__ float mx[MAXG], sm[MAXG];
+  extern __shared__ __align__(16) uint8_t sa_smem[];
+  uint16_t* ks = reinterpret_cast<uint16_t*>(sa_smem);            // [SLICE][RP]
+  uint16_t* vs = ks + SLICE * RP;                                  // [SLICE][RP]
+  float* qs = reinterpret_cast<float*>(vs + SLICE * RP);           // [MAXG][D]
+  float* ws = qs + MAXG * D;                                       // [MAXG][SLICE]
+  int* rows = reinterpret_cast<int*>(ws + MAXG * SLICE);           // [SLICE]
+  float* mx = reinterpret_cast<float*>(rows + SLICE);              // [MAXG]
+  float* sm = mx + MAXG;                                           // [MAXG]
   const int th = threadIdx.x;
-  for (int i = th; i < G * D; i += THREADS) {
-    const int g = i / D, dd = i % D;
-    qs[g][dd] = __uint_as_float((uint32_t)q[((size_t)t * Hq + hk * G + g) * D + dd] << 16) * scale;
-  }
   const int slot = split * SLICE + th;
   int p = -1;
   if (slot < P) {
@@ -60,42 +61,63 @@ __global__ void __launch_bounds__(sa::THREADS)
     }
   }
   rows[th] = p;
+  for (int i = th; i < G * D; i += THREADS) {
+    const int g = i / D, dd = i % D;
+    qs[g * D + dd] =
+        __uint_as_float((uint32_t)q[((size_t)t * Hq + hk * G + g) * D + dd] << 16) * scale;
+  }
+  __syncthreads();
+  // the slice's K and V rows into shared memory: every copy issued before
+  // the one wait (a chain of dependent loads would cost a DRAM round trip
+  // per row)
+  constexpr int CPR = D / 8;                 // 16-byte chunks per row
+  for (int c = th; c < SLICE * CPR; c += THREADS) {
+    const int i = c / CPR, j = c % CPR;
+    const int pr = rows[i];
+    if (pr < 0) continue;
+    const size_t off = ((size_t)pr * Hkv + hk) * D + 8 * j;
+    const uint32_t dk = smem_addr(ks + i * RP + 8 * j), dv = smem_addr(vs + i * RP + 8 * j);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dk), "l"(kc + off) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dv), "l"(vc + off) : "memory");
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   // scores of this thread's position for the G heads
   float s[MAXG];
 #pragma unroll
   for (int g = 0; g < MAXG; ++g) s[g] = 0.f;
   if (p >= 0) {
-    const uint4* kr = reinterpret_cast<const uint4*>(kc + ((size_t)p * Hkv + hk) * D);
+    const uint4* kr = reinterpret_cast<const uint4*>(ks + th * RP);
 #pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = __ldg(kr + c);
+    for (int c = 0; c < CPR; ++c) {
+      const uint4 v = kr[c];
       const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                           bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
 #pragma unroll
       for (int g = 0; g < MAXG; ++g) {
         if (g < G) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s[g] = fmaf(qs[g][8 * c + j], e[j], s[g]);
+          for (int j = 0; j < 8; ++j) s[g] = fmaf(qs[g * D + 8 * c + j], e[j], s[g]);
         }
       }
     }
   }
 #pragma unroll
   for (int g = 0; g < MAXG; ++g)
-    if (g < G) ws[g][th] = p >= 0 ? s[g] : -INFINITY;
+    if (g < G) ws[g * SLICE + th] = p >= 0 ? s[g] : -INFINITY;
   __syncthreads();
-  // per head: maximum and sum of exp(s - m) over the slice (warp g % 4 takes heads g)
+  // per head: maximum and sum of exp(s - m) over the slice
   const int warp = th >> 5, lane = th & 31;
   for (int g = warp; g < G; g += THREADS / 32) {
     float m = -INFINITY;
-    for (int i = lane; i < SLICE; i += 32) m = fmaxf(m, ws[g][i]);
+    for (int i = lane; i < SLICE; i += 32) m = fmaxf(m, ws[g * SLICE + i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     float l = 0.f;
     for (int i = lane; i < SLICE; i += 32) {
-      const float e = ws[g][i] == -INFINITY ? 0.f : __expf(ws[g][i] - m);
-      ws[g][i] = e;
+      const float x = ws[g * SLICE + i];
+      const float e = x == -INFINITY ? 0.f : __expf(x - m);
+      ws[g * SLICE + i] = e;
       l += e;
     }
 #pragma unroll
@@ -106,18 +128,17 @@ __global__ void __launch_bounds__(sa::THREADS)
     }
   }
   __syncthreads();
-  // o[g][d] = sum_p e[g][p] V[p][d]; thread = feature d (D <= 128 threads)
+  // o[g][d] = sum_p e[g][p] V[p][d]; thread = feature d
   if (th < D) {
     float o[MAXG];
 #pragma unroll
     for (int g = 0; g < MAXG; ++g) o[g] = 0.f;
     for (int i = 0; i < SLICE; ++i) {
-      const int pr = rows[i];
-      if (pr < 0) continue;
-      const float v = __uint_as_float((uint32_t)__ldg(vc + ((size_t)pr * Hkv + hk) * D + th) << 16);
+      if (rows[i] < 0) continue;
+      const float v = __uint_as_float((uint32_t)vs[i * RP + th] << 16);
 #pragma unroll
       for (int g = 0; g < MAXG; ++g)
-        if (g < G) o[g] = fmaf(ws[g][i], v, o[g]);
+        if (g < G) o[g] = fmaf(ws[g * SLICE + i], v, o[g]);
     }
 #pragma unroll
     for (int g = 0; g < MAXG; ++g)
@@ -128,6 +149,12 @@ __global__ void __launch_bounds__(sa::THREADS)
     part_ml[b] = mx[th];
     part_ml[b + 1] = sm[th];
   }
+}
+
+template <int D>
+constexpr int sparse_attn_smem() {
+  return 2 * sa::SLICE * (D + 8) * 2 + sa::MAXG * D * 4 + sa::MAXG * sa::SLICE * 4 +
+         sa::SLICE * 4 + 2 * sa::MAXG * 4;
 }
 
 template <int D>
@@ -166,12 +193,20 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* kc, const uint
   float* part_ml = part_o + (size_t)T * Hq * nsplit * D;
   const dim3 grid(nsplit, Hkv, T);
   if (D == 128) {
-    sparse_attn_split_kernel<128><<<grid, sa::THREADS, 0, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
-                                                               nsplit, scale, part_o, part_ml, err);
+    constexpr int sm = sparse_attn_smem<128>();
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_split_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    sparse_attn_split_kernel<128><<<grid, sa::THREADS, sm, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
+                                                                nsplit, scale, part_o, part_ml, err);
     sparse_attn_combine_kernel<128><<<T * Hq, 128, 0, s>>>(part_o, part_ml, nsplit, out);
   } else {
-    sparse_attn_split_kernel<64><<<grid, sa::THREADS, 0, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
-                                                              nsplit, scale, part_o, part_ml, err);
+    constexpr int sm = sparse_attn_smem<64>();
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_split_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    sparse_attn_split_kernel<64><<<grid, sa::THREADS, sm, s>>>(q, kc, vc, idx, L, Hq, Hkv, P,
+                                                               nsplit, scale, part_o, part_ml, err);
     sparse_attn_combine_kernel<64><<<T * Hq, 64, 0, s>>>(part_o, part_ml, nsplit, out);
   }
   return cudaGetLastError();
