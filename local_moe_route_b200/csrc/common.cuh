@@ -178,15 +178,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Bring the 2-D box at (x, y) into L2 only (no shared memory, no barrier):
-// a producer runs such prefetches ahead of its ring to deepen the pipeline.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 // L2 policies: data read once (streamed weights) leaves L2 first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

@@ -10,16 +10,16 @@
 // launch: the CTAs stay resident (cooperative launch, two per SM) and pass
 // through five phases separated by grid-wide barriers with bounded waits:
 //
-//   P0  router partial logits (items of 512 rows of W_r x 64 experts);
+//   P0  router partial logits (items of 128 rows of W_r x 64 experts);
 //       every CTA also converts x of all tokens to fp16 in shared memory;
 //   --- grid barrier
 //   P0b the logits, each summed once from the partials (spread over CTAs);
 //   --- grid barrier
-//   P1  every CTA sums the partials, picks each token's top k (exact ties to
+//   P1  every CTA reads the logits, picks each token's top k (exact ties to
 //       the lower expert index), the softmax weights, and groups the T*k
-//       slots by expert (counts, offsets, stable order) in its own shared
-//       memory: same inputs, same code, same result in every CTA, so no
-//       barrier follows;
+//       slots by expert (active experts, counts, first rows, stable order)
+//       in its own shared memory: same inputs, same code, same result in
+//       every CTA, so no barrier follows;
 //   P2  gate/up + SwiGLU: units of 16 weight rows of one expert, K split
 //       over the 8 consumer warps, both matrices streamed by TMA through a
 //       3-deep ring, B operand = x from shared memory; h to global (fp16);
@@ -28,6 +28,15 @@
 //       each stage carries the expert's h rows; output rows to global (fp32);
 //   --- grid barrier
 //   P4  combine: y_t = sum_j w_tj * row_(t,j), fp32 in slot order, bf16.
+//
+// Warp roles in P2 and P3: one producer warp (TMA), eight consumer warps
+// (matrix products) and one reducer warp.  The units are handed out
+// dynamically (a grid-wide counter, fetched one unit ahead by the producer),
+// so a CTA that streams faster takes more of them.  Consumer warps pass each
+// unit's partial sums to the reducer through a double buffer and go on to
+// the next unit at once; the reducer adds the warps' sums in a fixed order,
+// applies SwiGLU (P2) and stores.  Results do not depend on which CTA took
+// a unit.
 //
 // Matrix products use mma.sync m16n8k16 with fp16 operands: the weights as
 // exact integer codes (a nibble pair (i, i + 4) becomes an fp16 pair with one
@@ -45,7 +54,7 @@ namespace strata {
 namespace df {
 constexpr int MAXT = 4;                   // tokens per batch on this path
 constexpr int CONS = 8;                   // consumer warps
-constexpr int THREADS = (CONS + 1) * 32;  // + one producer warp
+constexpr int THREADS = (CONS + 2) * 32;  // + one producer warp + one reducer warp
 constexpr int ST = 3;                     // ring stages
 // A ring stage: gate/up: 16 rows x 1024 K of both matrices (16 KB) and their
 // scales (16 rows x 1024 / G groups each, at most 2 KB); down: 64 rows x
@@ -54,16 +63,20 @@ constexpr int ST = 3;                     // ring stages
 constexpr int SLOT = 18432;               // bytes per ring stage
 constexpr int P2_SC = 16384;              // offset of the gate/up scales in a stage
 constexpr int P3_H = 8192, P3_SC = 10240; // offsets of h and of the down scales
-constexpr int PF = 6;                     // stages the producer prefetches into L2 ahead
 constexpr int P2_ROWS = 16;               // gate/up unit: 16 rows, K split 8 ways
 constexpr int P2_KST = 1024;              // gate/up K per stage
 constexpr int P3_ROWS = 64;               // down unit: 4 row groups x 2 K halves
 constexpr int P3_KST = 256;               // down K per stage
-constexpr int P0_RS = 512;                // router rows per item
-constexpr int P0_MAXKS = 8;               // router K slices (d <= 4096)
+constexpr int P0_RS = 128;                // router rows per item
+constexpr int P0_MAXKS = 32;              // router K slices (d <= 4096)
 constexpr int XPT = 8;                    // 16-byte chunks of x per thread (T * d <= 8 * 8 * THREADS)
+constexpr int LPT = 16;                   // logits per thread in P1 (T * E <= 16 * THREADS)
 constexpr int MAXE = 1024, MAXK = 32;
 constexpr int MAXS = MAXT * MAXK;
+// A hand-off buffer to the reducer: [consumer warp][lane (g, t < 2)][8] fp32
+// (gate/up: rows g, g + 8 of gate then up, tokens 2t, 2t + 1; down: the first
+// four).  Lanes with t >= 2 hold tokens 4..7, which never exist here.
+constexpr int RED_BUF = CONS * 16 * 8;
 
 // Shared memory (offsets from a 1024-byte aligned base).  The x area holds
 // x of all tokens in fp16 ([T][d + 8], 16 bytes of padding per row so that
@@ -75,12 +88,11 @@ struct Smem {
     s.ring = 0;
     s.x = ST * SLOT;
     const int xb = ((T * (d + 8) * 2) + 1023) & ~1023;
-    s.red = s.x + xb;                            // [8 warps][32 lanes][8] fp32
-    s.bars = s.red + CONS * 32 * 8 * 4;
+    s.red = s.x + xb;                            // two hand-off buffers
+    s.bars = s.red + 2 * RED_BUF * 4;
     s.route = s.bars + 128;
-    // ids, w [MAXS]; counts, active [MAXE]; offsets [MAXE + 1]; rowtok,
-    // slotrow [MAXS]; misc [64]  (the scan scratch `pos` lives in the ring)
-    s.total = s.route + (2 * MAXS + 2 * MAXE + MAXE + 1 + 2 * MAXS + 64) * 4;
+    // ids, w, active, acnt, aoff, first, rowtok, slotrow [MAXS]; misc [64]
+    s.total = s.route + (8 * MAXS + 64) * 4;
     return s;
   }
 };
@@ -100,7 +112,8 @@ struct FusedArgs {
   float* logits;             // [T][E]
   uint16_t* h;               // [T*k][n] fp16, features interleaved within 8
   float* rows;               // [T*k][d] fp32
-  unsigned* sync;            // [4] zeroed before the launch
+  unsigned* sync;            // [8] zeroed before the launch: [0] barrier arrivals,
+                             // [2] abort, [4] / [5] gate-up / down unit counters
   unsigned* err;
   int T, d, E, k, n, G;
 };
@@ -123,66 +136,31 @@ __device__ __forceinline__ bool df_sync_grid(unsigned* sync, int b, unsigned* er
   return ok;
 }
 
-// Block-wide exclusive scan of v[0..n) in place (each thread takes a run of
-// consecutive entries), returning the total.  Uses tmp[0..32]; blockDim.x is
-// a multiple of 32 and at most 1024.
-__device__ int df_block_scan(int* v, int n, int* tmp) {
-  const int th = threadIdx.x, lane = th & 31, warp = th >> 5, nw = blockDim.x >> 5;
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int b0 = th * per;
-  int s = 0;
-  for (int i = 0; i < per; ++i)
-    if (b0 + i < n) s += v[b0 + i];
-  int incl = s;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  if (lane == 31) tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int wv = lane < nw ? tmp[lane] : 0;
-    int wi = wv;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, wi, off);
-      if (lane >= off) wi += o;
-    }
-    __syncwarp();
-    tmp[lane] = wi - wv;                         // exclusive prefix of the warp totals
-    if (lane == 31) tmp[32] = wi;                // grand total
-  }
-  __syncthreads();
-  int run = tmp[warp] + incl - s;
-  const int total = tmp[32];
-  for (int i = 0; i < per; ++i)
-    if (b0 + i < n) {
-      const int x = v[b0 + i];
-      v[b0 + i] = run;
-      run += x;
-    }
-  __syncthreads();
-  return total;
-}
-
 // ---------------------------------------------------------------------------
-// P0: partial router logits.  Item = (512 rows of W_r, 64 experts): thread
+// P0: partial router logits.  Item = (128 rows of W_r, 64 experts): thread
 // (row group rr = th / 8 of 32, 16-byte chunk c = th % 8 of 8 experts) loads
-// the chunk of rows rr, rr + 32, ... (16 rows) all at once, multiplies them
-// by x of those rows (staged per item in shared memory as fp32) and the 32
-// row groups are added in a fixed order.  Uses threads 0..255.
-//   scratch: >= 32 * MAXT * 64 + MAXT * 512 floats
+// the chunk of rows rr, rr + 32, rr + 64, rr + 96 at once, then x of the
+// item's rows is staged in shared memory as fp32, and the 32 row groups'
+// products are added in a fixed order.  Uses threads 0..255.
+//   scratch: >= 32 * MAXT * 64 + MAXT * P0_RS floats
 __device__ void df_router_partials(const FusedArgs& a, float* scratch) {
   using namespace df;
+  constexpr int RPT = P0_RS / 32;                         // rows per thread
   const int th = threadIdx.x;
   const int neb = (a.E + 63) / 64, nks = a.d / P0_RS;
   float* red = scratch;                                   // [32][MAXT][64]
-  float* xr = scratch + 32 * MAXT * 64;                   // [MAXT][512]
+  float* xr = scratch + 32 * MAXT * 64;                   // [MAXT][P0_RS]
+  const int c = th & 7, rr = th >> 3;
   for (int item = blockIdx.x; item < neb * nks; item += gridDim.x) {
     const int eb = item % neb, ks = item / neb;
     const int r0 = ks * P0_RS;
-    if (th < a.T * (P0_RS / 8)) {                         // one 16-byte chunk per thread
+    const int e0 = eb * 64 + c * 8;
+    const bool live = th < 256 && e0 < a.E;               // E % 8 == 0 on this path
+    uint4 w[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+      if (live) w[i] = ld_nc_v4(a.w_router + (size_t)(r0 + rr + 32 * i) * a.E + e0);
+    if (th < a.T * (P0_RS / 8)) {                         // one 16-byte chunk of x per thread
       const int t = th / (P0_RS / 8), j = th % (P0_RS / 8);
       const uint4 v = ld_nc_v4(a.x + (size_t)t * a.d + r0 + 8 * j);
       float* dst = xr + t * P0_RS + 8 * j;
@@ -191,20 +169,14 @@ __device__ void df_router_partials(const FusedArgs& a, float* scratch) {
     }
     __syncthreads();
     if (th < 256) {
-      const int c = th & 7, rr = th >> 3;
-      const int e0 = eb * 64 + c * 8;
       float acc[MAXT][8];
 #pragma unroll
       for (int t = 0; t < MAXT; ++t)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[t][j] = 0.f;
-      if (e0 < a.E) {                                     // E % 8 == 0 on this path
-        uint4 w[P0_RS / 32];
+      if (live) {
 #pragma unroll
-        for (int i = 0; i < P0_RS / 32; ++i)
-          w[i] = ld_nc_v4(a.w_router + (size_t)(r0 + rr + 32 * i) * a.E + e0);
-#pragma unroll
-        for (int i = 0; i < P0_RS / 32; ++i) {
+        for (int i = 0; i < RPT; ++i) {
           const float wv[8] = {bf16_lo(w[i].x), bf16_hi(w[i].x), bf16_lo(w[i].y), bf16_hi(w[i].y),
                                bf16_lo(w[i].z), bf16_hi(w[i].z), bf16_lo(w[i].w), bf16_hi(w[i].w)};
 #pragma unroll
@@ -226,7 +198,7 @@ __device__ void df_router_partials(const FusedArgs& a, float* scratch) {
     if (th < a.T * 64) {
       const int t = th / 64, l = th % 64;
       float sum = 0.f;
-      for (int g = 0; g < 32; ++g) sum += red[(g * MAXT + t) * 64 + l];
+      for (int gi = 0; gi < 32; ++gi) sum += red[(gi * MAXT + t) * 64 + l];
       const int ee = eb * 64 + l;
       if (ee < a.E) a.partial[((size_t)ks * a.T + t) * a.E + ee] = sum;
     }
@@ -272,15 +244,15 @@ __device__ bool df_load_x(const FusedArgs& a, uint16_t* xs) {
 // of the T*k slots by expert.  Every CTA computes it; CTA 0 writes the
 // optional outputs.
 struct Route {
-  int32_t* ids;      // [T*k]
-  float* w;          // [T*k]
-  int32_t* counts;   // [E]
-  int32_t* offsets;  // [E + 1]
-  int32_t* active;   // [n_active]
-  int32_t* pos;      // [E] scratch
+  int32_t* ids;      // [S] expert of each slot
+  float* w;          // [S] its softmax weight
+  int32_t* active;   // [n_active] experts with at least one slot, ascending
+  int32_t* acnt;     // [n_active] their slot counts
+  int32_t* aoff;     // [n_active] their first grouped row
+  int32_t* first;    // [S] scratch: slot is its expert's first
   int32_t* rowtok;   // [S] grouped row -> token
   int32_t* slotrow;  // [S] slot -> grouped row
-  int* misc;         // [0] n_active, [1..32] scan scratch
+  int* misc;         // [0] n_active
 };
 
 // P0b: the logits, each once: the K slices' partial sums in order, then the
@@ -308,9 +280,21 @@ __device__ void df_logits(const FusedArgs& a) {
 __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
   using namespace df;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nks = a.d / P0_RS, S = a.T * a.k;
+  const int S = a.T * a.k;
   // logits of every token (summed once, by all CTAs together, in P0b)
-  for (int i = threadIdx.x; i < a.T * a.E; i += blockDim.x) logit_s[i] = __ldcg(a.logits + i);
+  {
+    float v[LPT];                                      // every load first, then the stores
+#pragma unroll
+    for (int u = 0; u < LPT; ++u) {
+      const int i = threadIdx.x + u * blockDim.x;
+      v[u] = i < a.T * a.E ? __ldcg(a.logits + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < LPT; ++u) {
+      const int i = threadIdx.x + u * blockDim.x;
+      if (i < a.T * a.E) logit_s[i] = v[u];
+    }
+  }
   __syncthreads();
   // top k of each token by two warps: warp 2t + hf selects the k best of its
   // half of the experts (exact ties to the lower index, NaN never wins), then
@@ -425,30 +409,37 @@ __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
     }
   }
   __syncthreads();
-  // counts per expert and the rank of each slot among the slots of its expert
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-    int c = 0;
-    for (int s = 0; s < S; ++s) c += R.ids[s] == e;
-    R.counts[e] = c;
-    R.offsets[e] = c;
+  // grouping of the S <= 128 slots by expert, slot order within an expert:
+  // thread s scans the S ids once for its slot's rank among the slots of its
+  // expert, the slots of lower experts (its expert's first row) and its
+  // expert's count; the first slot of each expert then finds the expert's
+  // place among the active experts.
+  const int s = threadIdx.x;
+  int e = 0, rank = 0, less = 0, cnt = 0;
+  if (s < S) {
+    e = R.ids[s];
+    for (int s2 = 0; s2 < S; ++s2) {
+      const int e2 = R.ids[s2];
+      rank += (e2 == e) & (s2 < s);
+      less += e2 < e;
+      cnt += e2 == e;
+    }
+    R.slotrow[s] = less + rank;
+    R.rowtok[less + rank] = s / a.k;
+    R.first[s] = rank == 0;
   }
   __syncthreads();
-  df_block_scan(R.offsets, a.E, R.misc + 1);
-  if (threadIdx.x == 0) R.offsets[a.E] = S;
-  // active experts in ascending order: scan of the flags, then scatter
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) R.pos[e] = R.counts[e] > 0;
-  __syncthreads();
-  const int na = df_block_scan(R.pos, a.E, R.misc + 1);
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-    if (R.counts[e] > 0) R.active[R.pos[e]] = e;
-  if (threadIdx.x == 0) R.misc[0] = na;
-  for (int s = threadIdx.x; s < S; s += blockDim.x) {
-    const int e = R.ids[s];
-    int rank = 0;
-    for (int s2 = 0; s2 < s; ++s2) rank += R.ids[s2] == e;
-    const int row = R.offsets[e] + rank;
-    R.slotrow[s] = row;
-    R.rowtok[row] = s / a.k;
+  if (s < S && rank == 0) {
+    int j = 0;
+    for (int s2 = 0; s2 < S; ++s2) j += R.first[s2] & (R.ids[s2] < e);
+    R.active[j] = e;
+    R.acnt[j] = cnt;
+    R.aoff[j] = less;
+  }
+  if (s == 0) {
+    int na = 0;
+    for (int s2 = 0; s2 < S; ++s2) na += R.first[s2];
+    R.misc[0] = na;
   }
   __syncthreads();
 }
@@ -543,6 +534,30 @@ __device__ __forceinline__ int df_ilv(int f) {
   return (f & ~7) | (i < 4 ? 2 * i : 2 * (i - 4) + 1);
 }
 
+// A consumer warp hands its sums of unit u (u = -1: the phase's end) to the
+// reducer: hand-off number rc uses buffer rc % 2, free once the reducer has
+// finished hand-off rc - 2.  Warp 0 names the unit.  Returns false if the
+// wait gave up.
+__device__ __forceinline__ bool df_post(float* red, uint64_t* red_full, uint64_t* red_empty,
+                                        volatile int* red_unit, uint32_t& rc, int u,
+                                        const float* v, volatile int* abort, unsigned* err) {
+  using namespace df;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = rc & 1;
+  if (rc >= 2 && !mbar_wait_warp(&red_empty[b], ((rc >> 1) - 1) & 1, abort, err)) return false;
+  if (v != nullptr && (lane & 3) < 2) {
+    float4* p = reinterpret_cast<float4*>(red + b * RED_BUF +
+                                          (warp * 16 + (lane >> 2) * 2 + (lane & 3)) * 8);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  if (warp == 0 && lane == 0) red_unit[b] = u;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&red_full[b]);
+  ++rc;
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 template <int G>
 __global__ void __launch_bounds__(df::THREADS, 2)
@@ -564,19 +579,22 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   float* red = reinterpret_cast<float*>(smem + L.red);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + ST;
-  volatile int* flag = reinterpret_cast<volatile int*>(empty + ST);      // grid barrier result
+  uint64_t* red_full = empty + ST;          // [2] consumer warps -> reducer
+  uint64_t* red_empty = red_full + 2;       // [2] reducer -> consumer warps
+  volatile int* flag = reinterpret_cast<volatile int*>(red_empty + 2);  // grid barrier result
   volatile int* abort_flag = flag + 1;
+  volatile int* hdr = abort_flag + 1;       // [ST] unit of each ring stage
+  volatile int* red_unit = hdr + ST;        // [2] unit of each hand-off buffer
   Route R;
   {
     int32_t* r = reinterpret_cast<int32_t*>(smem + L.route);
     R.ids = r;
     R.w = reinterpret_cast<float*>(r + MAXS);
-    R.counts = r + 2 * MAXS;
-    R.active = R.counts + MAXE;
-    // after the P1 logits and the top-k candidates
-    R.pos = reinterpret_cast<int32_t*>(ring) + MAXT * MAXE + 2 * MAXT * 2 * MAXK;
-    R.offsets = R.active + MAXE;
-    R.rowtok = R.offsets + MAXE + 1;
+    R.active = r + 2 * MAXS;
+    R.acnt = R.active + MAXS;
+    R.aoff = R.acnt + MAXS;
+    R.first = R.aoff + MAXS;
+    R.rowtok = R.first + MAXS;
     R.slotrow = R.rowtok + MAXS;
     R.misc = R.slotrow + MAXS;
   }
@@ -588,6 +606,10 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CONS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&red_full[b], CONS);
+      mbar_init(&red_empty[b], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -613,41 +635,39 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   // the ring held generic-proxy data (P0, P1); the TMA writes into it next
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   const int n_active = ok ? R.misc[0] : 0;
-  const int S = a.T * a.k;
 
   uint32_t g = 0;                           // ring stage counter (both phases)
+  uint32_t rc = 0;                          // hand-off counter to the reducer (both phases)
+  // Units are handed out dynamically: CTA b starts with unit b, its producer
+  // then takes the next one from a grid-wide counter (fetched one unit
+  // ahead) and writes each stage's unit into hdr[stage]; a stage with unit
+  // -1 ends the phase.  Consumer warps hand each unit's partial sums to the
+  // reducer warp through one of two buffers and go straight on to the next
+  // unit; the reducer adds them in a fixed warp order and stores the results.
+
   // ---- P2: gate/up + SwiGLU, units (expert, 16 rows)
   const int FB2 = a.n / P2_ROWS, KS2 = a.d / P2_KST;
   const int units2 = n_active * FB2;
   if (warp == CONS) {
-    if (lane == 0) {
-      bool stop = false;
-      // stage q of this CTA's gate/up stream: unit blockIdx.x + (q / KS2) * gridDim.x, K block q % KS2
-      auto prefetch2 = [&](int q) {
-        const int u = blockIdx.x + (q / KS2) * (int)gridDim.x;
-        if (u >= units2) return;
-        const int kc = q % KS2;
-        const int wrow = R.active[u / FB2] * a.n + (u % FB2) * P2_ROWS;
-#pragma unroll
-        for (int b = 0; b < P2_KST / 256; ++b) {
-          tma_prefetch_2d(&map_wg, kc * (P2_KST / 2) + b * 128, wrow);
-          tma_prefetch_2d(&map_wu, kc * (P2_KST / 2) + b * 128, wrow);
-        }
-        tma_prefetch_2d(&map_sg, kc * (P2_KST / G), wrow);
-        tma_prefetch_2d(&map_su, kc * (P2_KST / G), wrow);
-      };
-      for (int q = 0; q < PF; ++q) prefetch2(q);
-      int q2 = 0;
-      for (int u = blockIdx.x; u < units2 && !stop; u += gridDim.x) {
-        const int e = R.active[u / FB2];
+    if (lane == 0 && ok) {
+      int u = blockIdx.x;
+      for (;;) {
+        const bool last = u >= units2;
+        const int nx = last ? 0 : (int)gridDim.x + (int)atomicAdd(&a.sync[4], 1u);
+        bool stop = false;
+        const int e = last ? 0 : R.active[u / FB2];
         const int wrow = e * a.n + (u % FB2) * P2_ROWS;
-        for (int kc = 0; kc < KS2; ++kc, ++g, ++q2) {
-          prefetch2(q2 + PF);
+        for (int kc = 0; kc < (last ? 1 : KS2); ++kc, ++g) {
           const int s = g % ST;
           if (g >= (uint32_t)ST &&
               !mbar_wait(&empty[s], ((g / ST) - 1) & 1, abort_flag, a.err)) {
             stop = true;
             break;
+          }
+          hdr[s] = last ? -1 : u;
+          if (last) {
+            mbar_arrive(&full[s]);
+            continue;
           }
           uint8_t* sl = ring + s * SLOT;
           constexpr int SG = P2_ROWS * (P2_KST / G) * 2;   // scale bytes per matrix
@@ -661,21 +681,32 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           tma_load_2d(sl + P2_SC, &map_sg, kc * (P2_KST / G), wrow, &full[s]);
           tma_load_2d(sl + P2_SC + SG, &map_su, kc * (P2_KST / G), wrow, &full[s]);
         }
+        if (stop || last) break;
+        u = nx;
       }
     }
-  } else {
+  } else if (warp < CONS) {
     const int ks = warp;                    // this warp's 128 K of each stage
     constexpr int SGR = P2_KST / G;         // scale groups per row in a stage
-    for (int u = blockIdx.x; u < units2; u += gridDim.x) {
-      const int e = R.active[u / FB2], fb = u % FB2;
-      const int cnt = R.counts[e], prow = R.offsets[e];
+    while (ok) {
+      int s = g % ST;
+      if (!mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) break;
+      const int u = hdr[s];
+      if (u < 0) {                          // the phase's end: release the stage, tell the reducer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        ++g;
+        df_post(red, red_full, red_empty, red_unit, rc, -1, nullptr, abort_flag, a.err);
+        break;
+      }
+      const int cnt = R.acnt[u / FB2], prow = R.aoff[u / FB2];
       const int tok = R.rowtok[prow + min(g8, cnt - 1)];
       const uint16_t* xr = xs + (size_t)tok * XP;
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       bool failed = false;
       for (int kc = 0; kc < KS2; ++kc, ++g) {
-        const int s = g % ST;
-        if (!mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) {
+        s = g % ST;
+        if (kc > 0 && !mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) {
           failed = true;
           break;
         }
@@ -709,58 +740,74 @@ __global__ void __launch_bounds__(df::THREADS, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
-      // the 8 warps' sums of the unit meet in shared memory (fixed order)
-      float4* rp = reinterpret_cast<float4*>(red + (warp * 32 + lane) * 8);
-      rp[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-      rp[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-      if (named_barrier_or(1, CONS * 32, failed || *abort_flag)) break;   // all warps alike
-      if (threadIdx.x < P2_ROWS * 8) {
-        const int r = threadIdx.x >> 3, col = threadIdx.x & 7;
-        const int ln = (r & 7) * 4 + (col >> 1), reg = (r >> 3) * 2 + (col & 1);
-        float gs = 0.f, us = 0.f;
+      if (failed) break;
+      const float v[8] = {acc[0][0], acc[0][1], acc[0][2], acc[0][3],
+                          acc[1][0], acc[1][1], acc[1][2], acc[1][3]};
+      if (!df_post(red, red_full, red_empty, red_unit, rc, u, v, abort_flag, a.err)) break;
+    }
+  } else {
+    // reducer: gate and up sums of 16 rows x cnt tokens; lane = (row r, token pair cp)
+    const int r = lane & 15, cp = lane >> 4;
+    uint32_t rr = rc;
+    while (ok) {
+      const int b = rr & 1;
+      if (!mbar_wait_warp(&red_full[b], (rr >> 1) & 1, abort_flag, a.err)) break;
+      const int u = red_unit[b];
+      if (u >= 0) {
+        const int fb = u % FB2;
+        const int cnt = R.acnt[u / FB2], prow = R.aoff[u / FB2];
+        const float* rb = red + b * RED_BUF + ((r & 7) * 2 + cp) * 8 + (r >> 3) * 2;
+        float gs[2] = {0.f, 0.f}, us[2] = {0.f, 0.f};
+#pragma unroll
         for (int w = 0; w < CONS; ++w) {
-          gs += red[(w * 32 + ln) * 8 + reg];
-          us += red[(w * 32 + ln) * 8 + 4 + reg];
+          const float2 gv = *reinterpret_cast<const float2*>(rb + w * 128);
+          const float2 uv = *reinterpret_cast<const float2*>(rb + w * 128 + 4);
+          gs[0] += gv.x; gs[1] += gv.y;
+          us[0] += uv.x; us[1] += uv.y;
         }
-        if (col < cnt) {
-          const float hv = gs / (1.0f + __expf(-gs)) * us;
-          if (f16_overflows(hv)) atomicOr(a.err, kErrRange);
-          a.h[(size_t)(prow + col) * a.n + df_ilv(fb * P2_ROWS + r)] = f16_bits(hv);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col = 2 * cp + c;
+          if (col < cnt) {
+            const float hv = gs[c] / (1.0f + __expf(-gs[c])) * us[c];
+            if (f16_overflows(hv)) atomicOr(a.err, kErrRange);
+            a.h[(size_t)(prow + col) * a.n + df_ilv(fb * P2_ROWS + r)] = f16_bits(hv);
+          }
         }
       }
-      named_barrier_sync(1, CONS * 32);     // red is reused by the next unit
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_empty[b]);
+      ++rr;
+      if (u < 0) break;
     }
+    rc = rr;
   }
   ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
 
   // ---- P3: down, units (expert, 64 rows): 4 row groups x 2 K halves
   const int FB3 = a.d / P3_ROWS, KS3 = a.n / P3_KST;
-  const int units3 = ok ? n_active * FB3 : 0;
+  const int units3 = n_active * FB3;
   if (warp == CONS) {
-    if (lane == 0) {
-      bool stop = false;
-      auto prefetch3 = [&](int q) {
-        const int u = blockIdx.x + (q / KS3) * (int)gridDim.x;
-        if (u >= units3) return;
-        const int kc = q % KS3;
-        const int e = R.active[u / FB3];
+    if (lane == 0 && ok) {
+      int u = blockIdx.x;
+      for (;;) {
+        const bool last = u >= units3;
+        const int nx = last ? 0 : (int)gridDim.x + (int)atomicAdd(&a.sync[5], 1u);
+        bool stop = false;
+        const int e = last ? 0 : R.active[u / FB3];
         const int wrow = e * a.d + (u % FB3) * P3_ROWS;
-        tma_prefetch_2d(&map_wd, kc * (P3_KST / 2), wrow);
-        if (kc == 0) tma_prefetch_2d(&map_sd, 0, wrow);
-      };
-      for (int q = 0; q < PF; ++q) prefetch3(q);
-      int q3 = 0;
-      for (int u = blockIdx.x; u < units3 && !stop; u += gridDim.x) {
-        const int e = R.active[u / FB3];
-        const int wrow = e * a.d + (u % FB3) * P3_ROWS;
-        const int prow = R.offsets[e];
-        for (int kc = 0; kc < KS3; ++kc, ++g, ++q3) {
-          prefetch3(q3 + PF);
+        const int prow = last ? 0 : R.aoff[u / FB3];
+        for (int kc = 0; kc < (last ? 1 : KS3); ++kc, ++g) {
           const int s = g % ST;
           if (g >= (uint32_t)ST &&
               !mbar_wait(&empty[s], ((g / ST) - 1) & 1, abort_flag, a.err)) {
             stop = true;
             break;
+          }
+          hdr[s] = last ? -1 : u;
+          if (last) {
+            mbar_arrive(&full[s]);
+            continue;
           }
           uint8_t* sl = ring + s * SLOT;
           mbar_arrive_expect_tx(&full[s], P3_ROWS * (P3_KST / 2) + MAXT * P3_KST * 2 +
@@ -769,20 +816,31 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           tma_load_2d(sl + P3_H, &map_h, kc * P3_KST, prow, &full[s]);
           tma_load_2d(sl + P3_SC, &map_sd, 0, wrow, &full[s]);     // the unit's scale rows
         }
+        if (stop || last) break;
+        u = nx;
       }
     }
-  } else {
+  } else if (warp < CONS) {
     const int rg = warp & 3, kh = warp >> 2;
     const int NG = a.n / G;                 // scale groups per down row
-    for (int u = blockIdx.x; u < units3; u += gridDim.x) {
-      const int e = R.active[u / FB3], fb = u % FB3;
-      const int cnt = R.counts[e], prow = R.offsets[e];
+    while (ok) {
+      int s = g % ST;
+      if (!mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) break;
+      const int u = hdr[s];
+      if (u < 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        ++g;
+        df_post(red, red_full, red_empty, red_unit, rc, -1, nullptr, abort_flag, a.err);
+        break;
+      }
+      const int cnt = R.acnt[u / FB3];
       const int hrow = g8 < cnt ? g8 : 0;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       bool failed = false;
       for (int kc = 0; kc < KS3; ++kc, ++g) {
-        const int s = g % ST;
-        if (!mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) {
+        s = g % ST;
+        if (kc > 0 && !mbar_wait_warp(&full[s], (g / ST) & 1, abort_flag, a.err)) {
           failed = true;
           break;
         }
@@ -811,21 +869,36 @@ __global__ void __launch_bounds__(df::THREADS, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
-      // second K half hands its sums to the first (fixed order: first + second)
-      float4* rp = reinterpret_cast<float4*>(red + (rg * 32 + lane) * 4);
-      if (kh == 1) *rp = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      if (named_barrier_or(1, CONS * 32, failed || *abort_flag)) break;   // all warps alike
-      if (kh == 0) {
-        const float4 o = *rp;
-        const float v[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};
+      if (failed) break;
+      const float v[8] = {acc[0], acc[1], acc[2], acc[3], 0.f, 0.f, 0.f, 0.f};
+      if (!df_post(red, red_full, red_empty, red_unit, rc, u, v, abort_flag, a.err)) break;
+    }
+  } else {
+    // reducer: 64 rows x cnt tokens, first K half + second K half (warps rg, rg + 4)
+    uint32_t rr = rc;
+    while (ok) {
+      const int b = rr & 1;
+      if (!mbar_wait_warp(&red_full[b], (rr >> 1) & 1, abort_flag, a.err)) break;
+      const int u = red_unit[b];
+      if (u >= 0) {
+        const int fb = u % FB3;
+        const int cnt = R.acnt[u / FB3], prow = R.aoff[u / FB3];
+        const float* rb = red + b * RED_BUF;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = 2 * t + (q & 1);
-          const int feat = fb * P3_ROWS + rg * 16 + g8 + (q >> 1) * 8;
-          if (col < cnt) a.rows[(size_t)(prow + col) * a.d + feat] = v[q];
+        for (int i = 0; i < 8; ++i) {
+          const int col = i >> 1, row = (i & 1) * 32 + lane;    // row of the unit's 64
+          if (col < cnt) {
+            const int rg = row >> 4, r16 = row & 15;
+            const int at = ((r16 & 7) * 2 + (col >> 1)) * 8 + (r16 >> 3) * 2 + (col & 1);
+            const float v = rb[rg * 128 + at] + rb[(rg + 4) * 128 + at];
+            a.rows[(size_t)(prow + col) * a.d + fb * P3_ROWS + row] = v;
+          }
         }
       }
-      named_barrier_sync(1, CONS * 32);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red_empty[b]);
+      ++rr;
+      if (u < 0) break;
     }
   }
   ok = df_sync_grid(a.sync, 3, a.err, flag, abort_flag) && ok;
@@ -836,15 +909,28 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.T * cpr; i += gridDim.x * blockDim.x) {
       const int tk = i / cpr, f0 = (i % cpr) * 8;
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int j = 0; j < a.k; ++j) {
-        const int sl = tk * a.k + j;
-        const float w = R.w[sl];
-        const float4* rp = reinterpret_cast<const float4*>(a.rows + (size_t)R.slotrow[sl] * a.d + f0);
-        const float4 r0 = __ldcg(rp), r1 = __ldcg(rp + 1);
-        v[0] = fmaf(w, r0.x, v[0]); v[1] = fmaf(w, r0.y, v[1]);
-        v[2] = fmaf(w, r0.z, v[2]); v[3] = fmaf(w, r0.w, v[3]);
-        v[4] = fmaf(w, r1.x, v[4]); v[5] = fmaf(w, r1.y, v[5]);
-        v[6] = fmaf(w, r1.z, v[6]); v[7] = fmaf(w, r1.w, v[7]);
+      // rows of 8 slots at a time: their loads are all issued before the sums
+      for (int j0 = 0; j0 < a.k; j0 += 8) {
+        float4 r[8][2];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < a.k) {
+            const float4* rp = reinterpret_cast<const float4*>(
+                a.rows + (size_t)R.slotrow[tk * a.k + j0 + u] * a.d + f0);
+            r[u][0] = __ldcg(rp);
+            r[u][1] = __ldcg(rp + 1);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < a.k) {
+            const float w = R.w[tk * a.k + j0 + u];
+            v[0] = fmaf(w, r[u][0].x, v[0]); v[1] = fmaf(w, r[u][0].y, v[1]);
+            v[2] = fmaf(w, r[u][0].z, v[2]); v[3] = fmaf(w, r[u][0].w, v[3]);
+            v[4] = fmaf(w, r[u][1].x, v[4]); v[5] = fmaf(w, r[u][1].y, v[5]);
+            v[6] = fmaf(w, r[u][1].z, v[6]); v[7] = fmaf(w, r[u][1].w, v[7]);
+          }
+        }
       }
       uint4 o;
       o.x = pack_bf16x2(v[0], v[1]);
@@ -854,7 +940,6 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       *reinterpret_cast<uint4*>(a.y + (size_t)tk * a.d + f0) = o;
     }
   }
-  (void)S;
 }
 
 // ---------------------------------------------------------------------------
@@ -863,7 +948,7 @@ bool decode_fused_fits(int T, int d, int E, int k, int n, int G) {
   if (T < 1 || T > MAXT || k > MAXK || E > MAXE) return false;
   if (G != 32 && G != 64 && G != 128) return false;
   if (d % P2_KST || d % P0_RS || d / P0_RS > P0_MAXKS || n % P3_KST || n % P2_ROWS ||
-      d % P3_ROWS || E % 8 || T * d > 8 * XPT * THREADS)
+      d % P3_ROWS || E % 8 || T * d > 8 * XPT * THREADS || T * E > LPT * THREADS)
     return false;
   // scale tiles by TMA: rows of at least 16 bytes, at most 256 groups, fitting the stage
   if ((P2_KST / G) % 8 || (n / G) % 8 || n / G > 256 || P3_SC + P3_ROWS * (n / G) * 2 > SLOT)
@@ -966,7 +1051,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, con
                      (uint64_t)(n / G) * 2, n / G, P3_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.sync, 0, 16, s);
+  cudaError_t e = cudaMemsetAsync(a.sync, 0, 32, s);   // barrier words, unit counters
   if (e != cudaSuccess) return e;
   const int smem = Smem::of(T, d).total + 1024;
   if (G == 32) return launch_fused_g<32>(maps, a, smem, s);
