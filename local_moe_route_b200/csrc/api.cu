@@ -367,7 +367,7 @@ strata_status_t strata_moe_expert_gemm_q4(strata_moe_op_t op, const uint16_t* a,
   const SchedRegions r = add_schedule(L, dims);
   const Region x16 = L.add(x16_bytes(dims));
   const Schedule sch = schedule_at(static_cast<uint8_t*>(ws), r);
-  if (launch_schedule(offsets, dims.E, dims.T * dims.k, sch, err, s) != cudaSuccess)
+  if (launch_schedule(offsets, dims.E, dims.T * dims.k, kTileRows, sch, err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
   return do_gemm(op == STRATA_OP_GATE_UP_SWIGLU ? 0 : 1, a, sorted_token, offsets, w0, w1,
                  row_scale, dims, out, sch,
@@ -430,7 +430,7 @@ strata_status_t strata_moe_forward(const uint16_t* x, const uint16_t* w_router, 
   if (launch_permute(ids, dims.T, dims.k, dims.E, counts, offsets, sorted_token, slot_row,
                      reinterpret_cast<int32_t*>(at(f.hist)), err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
-  if (launch_schedule(offsets, dims.E, dims.T * dims.k, sch, err, s) != cudaSuccess)
+  if (launch_schedule(offsets, dims.E, dims.T * dims.k, kTileRows, sch, err, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
   uint16_t* x16 = reinterpret_cast<uint16_t*>(at(f.x16));
   // h is internal here: it passes between the GEMMs in the interleaved

@@ -277,6 +277,84 @@ __device__ void df_logits(const FusedArgs& a) {
   }
 }
 
+// Order-preserving 32-bit key of a logit: larger float, larger key; NaN maps
+// to the key of -inf and -0 to that of +0 (so they compare as the float
+// comparison treats them in the selection).
+__device__ __forceinline__ uint32_t df_order_key(float f) {
+  if (f != f) f = -INFINITY;
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float df_key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Top k of token t by one warp: lane l holds experts l, l + 32, ... (NV per
+// lane, E <= 32 NV) as order-preserving keys (NaN as -inf, -0 as +0; absent
+// and taken entries as 0, below every key).  Each round every lane offers
+// its best entry (largest key, then lowest index), the warp takes the
+// largest key and, among the lanes offering it, the lowest expert index (two
+// warp reductions), and the owning lane clears that entry: exact ties go to
+// the lower expert index and NaN never wins.  Then the softmax over the k.
+template <int NV>
+__device__ __forceinline__ void df_topk(const FusedArgs& a, const Route& R, const float* logit_s,
+                                        int t, int lane) {
+  uint32_t key[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < a.E ? df_order_key(logit_s[t * a.E + e]) : 0u;
+  }
+  uint32_t my_key = 0, top = 0;
+  int my_i = 0;
+  for (int j = 0; j < a.k; ++j) {
+    // four independent chains over i mod 4, merged in index order
+    uint32_t bk[4] = {0u, 0u, 0u, 0u};
+    int bs[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = i & 3;
+      if (key[i] > bk[c]) {                 // the first of equal keys stays (lower index)
+        bk[c] = key[i];
+        bs[c] = i;
+      }
+    }
+#pragma unroll
+    for (int c = 1; c < 4; ++c) {
+      if (bk[c] > bk[0] || (bk[c] == bk[0] && bs[c] < bs[0])) {
+        bk[0] = bk[c];
+        bs[0] = bs[c];
+      }
+    }
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk[0]);
+    const int wi = __reduce_min_sync(0xffffffffu, bk[0] == wk ? lane + 32 * bs[0] : 0x7fffffff);
+    if ((wi & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (i == (wi >> 5)) key[i] = 0u;
+    }
+    if (j == 0) top = wk;
+    if (lane == j) {
+      my_key = wk;
+      my_i = wi;
+    }
+  }
+  const float my_v = df_key_value(my_key), top_v = df_key_value(top);
+  const float ex = (lane < a.k) ? expf(my_v - top_v) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < a.k) {
+    R.ids[t * a.k + lane] = my_i;
+    R.w[t * a.k + lane] = ex / sum;
+    if (blockIdx.x == 0) {
+      if (a.ids_out) a.ids_out[t * a.k + lane] = my_i;
+      if (a.w_out) a.w_out[t * a.k + lane] = ex / sum;
+    }
+  }
+}
+
 __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
   using namespace df;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,117 +374,10 @@ __device__ void df_route(const FusedArgs& a, const Route& R, float* logit_s) {
     }
   }
   __syncthreads();
-  // top k of each token by two warps: warp 2t + hf selects the k best of its
-  // half of the experts (exact ties to the lower index, NaN never wins), then
-  // warp 2t merges the two lists of k with the same order.  Any of the
-  // token's k best lies among its half's k best, so the merge is exact.
-  float* cand_v = logit_s + MAXT * MAXE;                  // [MAXT][2][MAXK]
-  int* cand_i = reinterpret_cast<int*>(cand_v + MAXT * 2 * MAXK);
-  const int half = (a.E + 1) / 2;
-  if (warp < 2 * a.T) {
-    const int t = warp >> 1, hf = warp & 1;
-    const int lo = hf * half, hi = min(a.E, lo + half);
-    float v[MAXE / 64];
-    uint32_t taken = 0;
-#pragma unroll
-    for (int i = 0; i < MAXE / 64; ++i) {
-      const int e = lo + lane + 32 * i;
-      v[i] = -INFINITY;
-      if (e < hi) v[i] = logit_s[t * a.E + e];
-      else taken |= 1u << i;
-    }
-    for (int j = 0; j < a.k; ++j) {
-      float best = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < MAXE / 64; ++i) {
-        if (!((taken >> i) & 1u)) {
-          const float c = (v[i] != v[i]) ? -INFINITY : v[i];
-          const int e = lo + lane + 32 * i;
-          if (c > best || (c == best && e < bi)) {
-            best = c;
-            bi = e;
-          }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ob > best || (ob == best && oi < bi)) {
-          best = ob;
-          bi = oi;
-        }
-      }
-      if (bi != 0x7fffffff && ((bi - lo) & 31) == lane) taken |= 1u << ((bi - lo) >> 5);
-      if (lane == 0) {
-        cand_v[(t * 2 + hf) * MAXK + j] = best;
-        cand_i[(t * 2 + hf) * MAXK + j] = bi;
-      }
-    }
-  }
-  __syncthreads();
+  // top k of each token by one warp (warp t)
   if (warp < a.T) {
-    const int t = warp;
-    // the 2k candidates, lane l holding numbers l and l + 32 (candidate c is
-    // number c of the first half's list for c < k, else c - k of the second)
-    float cv[2];
-    int ci[2];
-    bool taken[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = lane + 32 * u;
-      cv[u] = -INFINITY;
-      ci[u] = 0x7fffffff;
-      if (c < 2 * a.k) {
-        const int hf = c < a.k ? 0 : 1, j = c < a.k ? c : c - a.k;
-        cv[u] = cand_v[(t * 2 + hf) * MAXK + j];
-        ci[u] = cand_i[(t * 2 + hf) * MAXK + j];
-      }
-      taken[u] = ci[u] == 0x7fffffff;
-    }
-    float my_v = 0.f, top = 0.f;
-    int my_i = 0;
-    for (int j = 0; j < a.k; ++j) {
-      float best = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (!taken[u] && (cv[u] > best || (cv[u] == best && ci[u] < bi))) {
-          best = cv[u];
-          bi = ci[u];
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ob > best || (ob == best && oi < bi)) {
-          best = ob;
-          bi = oi;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-        if (!taken[u] && ci[u] == bi) taken[u] = true;
-      if (j == 0) top = best;
-      if (lane == j) {
-        my_v = best;
-        my_i = bi;
-      }
-    }
-    const float ex = (lane < a.k) ? expf(my_v - top) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane < a.k) {
-      R.ids[t * a.k + lane] = my_i;
-      R.w[t * a.k + lane] = ex / sum;
-      if (blockIdx.x == 0) {
-        if (a.ids_out) a.ids_out[t * a.k + lane] = my_i;
-        if (a.w_out) a.w_out[t * a.k + lane] = ex / sum;
-      }
-    }
+    if (a.E <= 512) df_topk<16>(a, R, logit_s, warp, lane);
+    else df_topk<MAXE / 32>(a, R, logit_s, warp, lane);
   }
   __syncthreads();
   // grouping of the S <= 128 slots by expert, slot order within an expert:

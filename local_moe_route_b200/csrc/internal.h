@@ -18,7 +18,7 @@ constexpr int kStreamMaxTokens = 8;
 
 // Per-expert work lists derived from offsets (built on the device).
 struct Schedule {
-  int32_t* tile_prefix;   // [E+1]  tiles of kTileRows rows before expert e; [E] = total
+  int32_t* tile_prefix;   // [E+1]  tiles before expert e; [E] = total
   int4* tile_table;       // [max_tiles] (expert, first grouped row, rows, 0)
   int32_t* active;        // [E]   experts with at least one row, ascending
   int32_t* n_active;      // [1]
@@ -52,8 +52,10 @@ int router_ksplit(int T, int d, int E);
 cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_token, int32_t* slot_row,
                            int32_t* hist, unsigned* err, cudaStream_t s);
-cudaError_t launch_schedule(const int32_t* offsets, int E, int S, Schedule sch, unsigned* err,
-                            cudaStream_t s);
+// tile_rows: token rows per tile of the tensor-core GEMM that follows
+// (kTileRows); max_tiles bounds the table for tiles of at least kTileRows.
+cudaError_t launch_schedule(const int32_t* offsets, int E, int S, int tile_rows, Schedule sch,
+                            unsigned* err, cudaStream_t s);
 
 // ---- expert GEMMs
 struct GemmProblem {
@@ -75,6 +77,10 @@ struct GemmProblem {
   unsigned* err;
 };
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
+// Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]), features interleaved
+// within groups of 8 (0, 4, 1, 5, 2, 6, 3, 7).
+cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* sorted_token, int T, int d,
+                                   int S, uint16_t* xs, unsigned* err, cudaStream_t s);
 cudaError_t launch_gemm_stream(const GemmProblem& p, const Schedule& sch, cudaStream_t s);
 // Decode batches with K % 256 == 0, N % 64 == 0 and a group of 32, 64 or 128
 // (weights staged by TMA); cudaErrorNotSupported for other shapes.

@@ -133,14 +133,14 @@ cudaError_t launch_permute(const int32_t* ids, int T, int k, int E, int32_t* cou
   return cudaGetLastError();
 }
 
-// Work lists for the expert GEMMs: tiles of kTileRows rows per expert, the
+// Work lists for the expert GEMMs: tiles of tile_rows rows per expert, the
 // table that maps a global tile index to (expert, tile in expert), and the
 // ascending list of experts that received rows.  One block of 1024 threads.
 // Offsets that are not a non-decreasing sequence from 0 to S are reported
 // through the check word and leave every work list empty.
 __global__ void __launch_bounds__(1024)
-    schedule_kernel(const int32_t* __restrict__ offsets, int E, int S, Schedule sch,
-                    unsigned* err) {
+    schedule_kernel(const int32_t* __restrict__ offsets, int E, int S, int tile_rows,
+                    Schedule sch, unsigned* err) {
   const int e = threadIdx.x;
   bool bad = false;
   if (e < E) bad = offsets[e] < 0 || offsets[e + 1] < offsets[e] || offsets[e + 1] > S;
@@ -148,15 +148,15 @@ __global__ void __launch_bounds__(1024)
   bad = __syncthreads_or(bad);
   if (bad && e == 0) atomicOr(err, kErrIndex);
   const int cnt = (e < E && !bad) ? offsets[e + 1] - offsets[e] : 0;
-  const int tiles = (cnt + kTileRows - 1) / kTileRows;
+  const int tiles = (cnt + tile_rows - 1) / tile_rows;
   int total_tiles, total_active;
   const int tp = block_exclusive_scan(tiles, &total_tiles);
   const int ap = block_exclusive_scan(cnt > 0 ? 1 : 0, &total_active);
   if (e < E) {
     sch.tile_prefix[e] = tp;
     for (int j = 0; j < tiles; ++j) {
-      const int p0 = offsets[e] + j * kTileRows;
-      sch.tile_table[tp + j] = make_int4(e, p0, min(kTileRows, cnt - j * kTileRows), 0);
+      const int p0 = offsets[e] + j * tile_rows;
+      sch.tile_table[tp + j] = make_int4(e, p0, min(tile_rows, cnt - j * tile_rows), 0);
     }
     if (cnt > 0) sch.active[ap] = e;
   }
@@ -166,9 +166,9 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-cudaError_t launch_schedule(const int32_t* offsets, int E, int S, Schedule sch, unsigned* err,
-                            cudaStream_t s) {
-  schedule_kernel<<<1, 1024, 0, s>>>(offsets, E, S, sch, err);
+cudaError_t launch_schedule(const int32_t* offsets, int E, int S, int tile_rows, Schedule sch,
+                            unsigned* err, cudaStream_t s) {
+  schedule_kernel<<<1, 1024, 0, s>>>(offsets, E, S, tile_rows, sch, err);
   return cudaGetLastError();
 }
 
