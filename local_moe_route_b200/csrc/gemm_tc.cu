@@ -22,7 +22,9 @@
 //
 // Warp roles (480 threads, persistent, one CTA per SM):
 //   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
-//                swizzle) into an 8-deep ring
+//                swizzle) into an 8-deep ring, and of the group scales: one
+//                block of 8 groups of both slots' rows (16 B per row) every
+//                8 G / 64 stages into a two-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
 //   warp 2       token rows into a 4-deep ring, one TMA tile of 128 rows per
 //                stage: the down projection reads h, whose rows are already
@@ -32,10 +34,14 @@
 //                token-order copy with tile::gather4 copies instead, 32 per
 //                stage, left the MMA waiting on them 64% of the time and
 //                doubled the kernel's time at T = 6144.)
-//   warps 3-10   two dequantising warpgroups taking alternate stages; thread
-//                = weight row; fp16 pairs go to TMEM with tcgen05.st; each
-//                thread loads its row's group scales one block of groups
-//                ahead into registers
+//   warps 3-10   two (down: three) dequantising warpgroups taking the
+//                stages round-robin; thread = weight row; fp16 pairs go to
+//                TMEM with tcgen05.st; at each scale block a thread copies its
+//                rows' 8 scales into registers and frees the ring slot.  (When
+//                K / G is not a multiple of 8 the rows' scales are loaded from
+//                global memory one block ahead instead.  Those register loads
+//                cost the large workload about 6%: a thread's next release of
+//                a ring slot waited for its load in flight.)
 //   warps 11-14  epilogue: TMEM -> registers -> SwiGLU or row scale -> fp16,
 //                transposed through shared memory into whole-row stores
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/128, four A
@@ -48,6 +54,7 @@
 // goes into the mantissa of 1024.0 (giving 1032 + q), one fma subtracts 1032
 // exactly, one fp16 multiply by the fp16 group scale rounds once.
 #include "common.cuh"
+#include "dequant.cuh"
 #include "internal.h"
 
 namespace strata {
@@ -61,6 +68,10 @@ constexpr int A_ST = 4;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
 constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output feature)
+// Group scales by TMA (when K / G is a multiple of 8): blocks of 8 groups of
+// both slots' 128 rows (16 bytes per row and slot) in a two-deep ring.
+constexpr int SC_GROUPS = 8;
+constexpr int SC_BYTES = 2 * BM * SC_GROUPS * 2;   // 4 KB per block
 
 constexpr int W_TMA = 0, W_MMA = 1, W_BTMA = 2, W_DQ = 3;
 // Dequantising warpgroups take the stages round-robin: two for gate/up,
@@ -85,8 +96,9 @@ struct Lay {
   static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;    // [B_ST][B_BYTES]
   static constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;            // [slices * BM][STG_PITCH]
   static constexpr int STG_BYTES = (OP == 0 ? 1 : 2) * BM * STG_PITCH * 2;
-  static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
-  static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2;
+  static constexpr int SC_OFF = STG_OFF + STG_BYTES;                 // [2][2][BM][8] fp16
+  static constexpr int BAR_OFF = SC_OFF + 2 * SC_BYTES;
+  static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = 1024 + MISC_OFF + 64;
 };
@@ -140,52 +152,6 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int u, int FB) {
   return U;
 }
 
-// Packed int4 codes hold element i of a group of 8 in nibble i as a two's
-// complement value q in [-8, 7].  XOR with 0x8 turns a nibble into q + 8, and
-// placing q + 8 in the low mantissa bits of fp16 1024.0 gives 1032 + q
-// exactly; subtracting 1032 leaves q and one fp16 multiply gives the weight
-// RNE_fp16(q * s).
-
-// 8 codes -> 4 fp16 pairs in natural K order: pair i = (element 2i, 2i+1).
-__device__ __forceinline__ void dequant8(uint32_t w, uint32_t sc2, uint32_t* r) {
-  const uint32_t wx = w ^ 0x88888888u;
-  const uint32_t wx4 = wx >> 4;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    // byte i of wx (element 2i in its low nibble) to the low half, byte i of
-    // wx >> 4 (element 2i+1 in its low nibble) to the high half
-    const uint32_t t = __byte_perm(wx, wx4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
-    const uint32_t v = (t & 0x000F000Fu) | 0x64006400u;        // 1032 + q, both halves
-    uint32_t qv, o;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(qv) : "r"(v), "r"(0x3C003C00u), "r"(0xE408E408u));
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o) : "r"(qv), "r"(sc2));
-    r[i] = o;
-  }
-}
-
-// 8 codes -> 4 fp16 pairs in the interleaved K order (0,4), (1,5), (2,6),
-// (3,7): each pair comes out of one mask-and-or, with no byte permute.  The
-// operand it is multiplied with must use the same order within each group
-// of 8 (the grouped fp16 copy of x is written that way).
-__device__ __forceinline__ void dequant8_interleaved(uint32_t w, uint32_t sc2, uint32_t* r) {
-  const uint32_t wx = w ^ 0x88888888u;
-  const uint32_t wx8 = wx >> 8;
-  const uint32_t v0 = (wx & 0x000F000Fu) | 0x64006400u;   // 1024 + (q + 8):   elements 0, 4
-  const uint32_t v1 = (wx & 0x00F000F0u) | 0x64006400u;   // 1024 + 16(q + 8): elements 1, 5
-  const uint32_t v2 = (wx8 & 0x000F000Fu) | 0x64006400u;  // elements 2, 6
-  const uint32_t v3 = (wx8 & 0x00F000F0u) | 0x64006400u;  // elements 3, 7
-  uint32_t q0, q1, q2, q3;
-  // 1024 + (q + 8) - 1032 = q;  (1024 + 16(q + 8)) / 16 - 72 = q  (all exact)
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q0) : "r"(v0), "r"(0x3C003C00u), "r"(0xE408E408u));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q1) : "r"(v1), "r"(0x2C002C00u), "r"(0xD480D480u));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q2) : "r"(v2), "r"(0x3C003C00u), "r"(0xE408E408u));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(q3) : "r"(v3), "r"(0x2C002C00u), "r"(0xD480D480u));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(q0), "r"(sc2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[1]) : "r"(q1), "r"(sc2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(q2), "r"(sc2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r[3]) : "r"(q3), "r"(sc2));
-}
-
 // Gate/up B operand: xs[p] = fp16(x[sorted_token[p]]) for the S grouped rows,
 // with K interleaved within each group of 8 (0, 4, 1, 5, 2, 6, 3, 7) to match
 // dequant8_interleaved.  Out-of-range token indices are reported (kErrIndex)
@@ -228,11 +194,22 @@ __global__ void __launch_bounds__(256)
   if (bad) atomicOr(err, kErrIndex);
 }
 
-template <int OP, bool ILV>
+cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* sorted_token, int T, int d,
+                                   int S, uint16_t* xs, unsigned* err, cudaStream_t s) {
+  long blocks = (S + 7) / 8;                       // 8 rows (warps) per block
+  if (blocks > 16L * sm_count()) blocks = 16L * sm_count();
+  if (blocks < 1) return cudaSuccess;
+  gather_rows_f16_kernel<<<(int)blocks, 256, 0, s>>>(x, sorted_token, T, d, S, xs, err);
+  return cudaGetLastError();
+}
+
+template <int OP, bool ILV, bool STMA>
 __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
                           const __grid_constant__ CUtensorMap map_q1,
-                          const __grid_constant__ CUtensorMap map_b, const TcArgs args) {
+                          const __grid_constant__ CUtensorMap map_b,
+                          const __grid_constant__ CUtensorMap map_s0,
+                          const __grid_constant__ CUtensorMap map_s1, const TcArgs args) {
   using namespace tc;
   using Ly = Lay<OP>;
   constexpr int B_ST = Ly::B_ST;
@@ -251,6 +228,9 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   uint64_t* a_empty = a_full + A_ST;
   uint64_t* acc_full = a_empty + A_ST;
   uint64_t* acc_empty = acc_full + 1;
+  uint64_t* sc_full = acc_empty + 1;           // [2] scale blocks
+  uint64_t* sc_empty = sc_full + 2;            // [2]
+  uint8_t* sSc = smem + Ly::SC_OFF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::MISC_OFF + 4);
 
@@ -275,6 +255,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, BM);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sc_full[b], 1);
+      mbar_init(&sc_empty[b], Roles<OP>::NWG * BM);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -282,6 +266,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     prefetch_tmap(&map_q0);
     if (OP == 0) prefetch_tmap(&map_q1);
     prefetch_tmap(&map_b);
+    if (STMA) {
+      prefetch_tmap(&map_s0);
+      if (OP == 0) prefetch_tmap(&map_s1);
+    }
   }
   if (warp == W_MMA) tmem_alloc(tmem_holder, TMEM_COLS);
   tc_fence_before();
@@ -298,11 +286,28 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     // -------------------------------------------------------------- TMA producer
     if (lane == 0) {
       const CUtensorMap* map_slot1 = OP == 0 ? &map_q1 : &map_q0;
-      uint32_t g = 0;
+      const CUtensorMap* smap_slot1 = OP == 0 ? &map_s1 : &map_s0;
+      const int SPB = SC_GROUPS * G / BK;     // stages per scale block (4, 8 or 16)
+      uint32_t g = 0, gs = 0;
       bool stop = false;
       for (int i = 0; i < my_units && !stop; ++i) {
         const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
         for (int kb = 0; kb < KB; ++kb, ++g) {
+          if (STMA && kb % SPB == 0) {
+            // the scale block of the next SPB stages: rows of both slots,
+            // groups kb * BK / G .. + 8 (x coordinate a multiple of 8)
+            const int ss = gs & 1;
+            if (gs >= 2 &&
+                !mbar_wait(&sc_empty[ss], ((gs >> 1) - 1) & 1, abort_flag, args.err)) {
+              stop = true;
+              break;
+            }
+            mbar_arrive_expect_tx(&sc_full[ss], SC_BYTES);
+            tma_load_2d(sSc + ss * SC_BYTES, &map_s0, kb * BK / G, U.wrow[0], &sc_full[ss]);
+            tma_load_2d(sSc + ss * SC_BYTES + SC_BYTES / 2, smap_slot1, kb * BK / G, U.wrow[1],
+                        &sc_full[ss]);
+            ++gs;
+          }
           const int s = g % RAW_ST;
           if (g >= (uint32_t)RAW_ST &&
               !mbar_wait(&raw_empty[s], ((g / RAW_ST) - 1) & 1, abort_flag, args.err)) {
@@ -394,6 +399,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     // aligned 16-, 8-, 4- or 2-byte load).  The block after the one in use
     // is always in flight: a load has the time of SB groups to arrive.
     const int SB = (KG & 7) == 0 ? 8 : (KG & 3) == 0 ? 4 : (KG & 1) == 0 ? 2 : 1;
+    uint32_t gsr = 0;                        // scale blocks taken from the ring (STMA)
     int4 te_c = make_int4(0, 0, 0, 0), te_n = make_int4(0, 0, 0, 0);
     int unit_c = -1;
     auto tile_of = [&](int i) { return ld_nc_s4(args.tile_table + (blockIdx.x + i * gridDim.x) / FB); };
@@ -437,7 +443,28 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     for (int g = wg; g < total_stages; g += NWG) {
       const int grp0 = (kb * BK) >> g_shift;
       const int key = (iu << 16) | (grp0 & ~(SB - 1));
-      if (key != key_c) {
+      if (STMA && key != key_c) {
+        // this block's scales of both slots from the TMA ring into
+        // registers; the slot is released at once
+        const int ss = gsr & 1;
+        if (!mbar_wait(&sc_full[ss], (gsr >> 1) & 1, abort_flag, args.err)) break;
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+          blk_c[mm] = *reinterpret_cast<const uint4*>(sSc + ss * SC_BYTES + mm * (SC_BYTES / 2) +
+                                                       r * 16);
+        fence_proxy_async_smem();              // the loads before the next TMA write
+        mbar_arrive(&sc_empty[ss]);
+        ++gsr;
+        key_c = key;
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm) {
+          const uint4 b = blk_c[mm];
+          big_scale |= __vcmpgtu2(b.x & 0x7FFF7FFFu, 0x6FFF6FFFu) |
+                       __vcmpgtu2(b.y & 0x7FFF7FFFu, 0x6FFF6FFFu) |
+                       __vcmpgtu2(b.z & 0x7FFF7FFFu, 0x6FFF6FFFu) |
+                       __vcmpgtu2(b.w & 0x7FFF7FFFu, 0x6FFF6FFFu);
+        }
+      } else if (!STMA && key != key_c) {
         if (iu != unit_c) {
           te_c = (unit_c >= 0 && iu == unit_c + 1) ? te_n : tile_of(iu);
           unit_c = iu;
@@ -655,7 +682,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   }
 }
 
-template <int OP, bool ILV>
+template <int OP, bool ILV, bool STMA>
 static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
   CUtensorMap m0, m1;
   const uint64_t rows = (uint64_t)p.E * p.N;
@@ -676,8 +703,23 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
                      tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // group scales [E * N][K / G] fp16, blocks of 8 groups x 128 rows
+  CUtensorMap ms0 = m0, ms1 = m0;
+  if (STMA) {
+    const int KG = p.K / p.G;
+    if (encode_tmap_2d(&ms0, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.s0, KG, rows, (uint64_t)KG * 2,
+                       tc::SC_GROUPS, tc::BM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    ms1 = ms0;
+    if (OP == 0 &&
+        encode_tmap_2d(&ms1, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.s1, KG, rows, (uint64_t)KG * 2,
+                       tc::SC_GROUPS, tc::BM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   {
-    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP, ILV>,
+    cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP, ILV, STMA>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          tc::Lay<OP>::SMEM);
     if (e != cudaSuccess) return e;
@@ -709,15 +751,26 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-  moe_gemm_q4_tc_kernel<OP, ILV><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP>::SMEM, s>>>(m0, m1,
-                                                                                        mb, a);
+  moe_gemm_q4_tc_kernel<OP, ILV, STMA><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP>::SMEM, s>>>(
+      m0, m1, mb, ms0, ms1, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
-  if (p.op == 0)
-    return p.h_interleaved ? launch_tc_impl<0, true>(p, sch, s) : launch_tc_impl<0, false>(p, sch, s);
-  return p.h_interleaved ? launch_tc_impl<1, true>(p, sch, s) : launch_tc_impl<1, false>(p, sch, s);
+  // scales by TMA when a row's K / G groups make whole 16-byte blocks
+  const bool st = (p.K / p.G) % tc::SC_GROUPS == 0;
+  if (p.op == 0) {
+    if (st)
+      return p.h_interleaved ? launch_tc_impl<0, true, true>(p, sch, s)
+                             : launch_tc_impl<0, false, true>(p, sch, s);
+    return p.h_interleaved ? launch_tc_impl<0, true, false>(p, sch, s)
+                           : launch_tc_impl<0, false, false>(p, sch, s);
+  }
+  if (st)
+    return p.h_interleaved ? launch_tc_impl<1, true, true>(p, sch, s)
+                           : launch_tc_impl<1, false, true>(p, sch, s);
+  return p.h_interleaved ? launch_tc_impl<1, true, false>(p, sch, s)
+                         : launch_tc_impl<1, false, false>(p, sch, s);
 }
 
 }  // namespace strata

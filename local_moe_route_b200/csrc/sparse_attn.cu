@@ -12,12 +12,13 @@
 // Small query batches (decode, speculative verify) are bound by the bytes of
 // the selected rows, 2 * Hkv * D * 2 bytes per position per query.  Two
 // kernels, split-K style:
-//   1. one CTA per (query, KV head, slice of 128 index slots): the slice's
+//   1. one CTA per (query, KV head, slice of 64 index slots): the slice's
 //      selected K and V rows are copied into shared memory (cp.async, all
-//      issued before one wait); every thread takes one slot and forms the
-//      scores of the G query heads that share the KV head; the slice's
-//      softmax maximum and sum per head stay in shared memory; thread d
-//      accumulates sum_p exp(s - m) V[p][d] over the slice, fp32;
+//      issued before one wait); two threads take one slot, each forming the
+//      scores of the G query heads that share the KV head over half of D,
+//      and add them; the slice's softmax maximum and sum per head stay in
+//      shared memory; thread d accumulates sum_p exp(s - m) V[p][d] over the
+//      slice, fp32;
 //   2. one CTA per (query, head) rescales and adds the slices' partial sums
 //      (max-subtracted exponentials, fixed order) and rounds to bf16.
 #include "common.cuh"
@@ -26,9 +27,10 @@
 namespace strata {
 
 namespace sa {
-constexpr int SLICE = 128;     // index slots per CTA (one per thread)
+constexpr int SLICE = 64;      // index slots per CTA (two threads per slot for the scores)
 constexpr int THREADS = 128;
 constexpr int MAXG = 16;       // query heads per KV head
+constexpr int MAXSPLIT = 1024; // slices per query (P <= 65536)
 }  // namespace sa
 
 template <int D>
@@ -51,16 +53,18 @@ __global__ void __launch_bounds__(sa::THREADS)
   float* mx = reinterpret_cast<float*>(rows + SLICE);              // [MAXG]
   float* sm = mx + MAXG;                                           // [MAXG]
   const int th = threadIdx.x;
-  const int slot = split * SLICE + th;
-  int p = -1;
-  if (slot < P) {
-    p = idx[(size_t)t * P + slot];
-    if (p >= L) {
-      atomicOr(err, kErrIndex);
-      p = -1;
+  if (th < SLICE) {
+    const int slot = split * SLICE + th;
+    int p = -1;
+    if (slot < P) {
+      p = idx[(size_t)t * P + slot];
+      if (p >= L) {
+        atomicOr(err, kErrIndex);
+        p = -1;
+      }
     }
+    rows[th] = p;
   }
-  rows[th] = p;
   for (int i = th; i < G * D; i += THREADS) {
     const int g = i / D, dd = i % D;
     qs[g * D + dd] =
@@ -82,29 +86,36 @@ __global__ void __launch_bounds__(sa::THREADS)
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
-  // scores of this thread's position for the G heads
+  // scores of slot th / 2 for the G heads: the two threads of a slot take
+  // one half of D each and add their sums (fixed order: lower half first)
+  const int sl = th >> 1, hf = th & 1;
+  const int p = rows[sl];
   float s[MAXG];
 #pragma unroll
   for (int g = 0; g < MAXG; ++g) s[g] = 0.f;
   if (p >= 0) {
-    const uint4* kr = reinterpret_cast<const uint4*>(ks + th * RP);
+    const uint4* kr = reinterpret_cast<const uint4*>(ks + sl * RP) + hf * (CPR / 2);
 #pragma unroll 4
-    for (int c = 0; c < CPR; ++c) {
+    for (int c = 0; c < CPR / 2; ++c) {
       const uint4 v = kr[c];
       const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                           bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+      const int d0 = (hf * (CPR / 2) + c) * 8;
 #pragma unroll
       for (int g = 0; g < MAXG; ++g) {
         if (g < G) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s[g] = fmaf(qs[g * D + 8 * c + j], e[j], s[g]);
+          for (int j = 0; j < 8; ++j) s[g] = fmaf(qs[g * D + d0 + j], e[j], s[g]);
         }
       }
     }
   }
 #pragma unroll
-  for (int g = 0; g < MAXG; ++g)
-    if (g < G) ws[g * SLICE + th] = p >= 0 ? s[g] : -INFINITY;
+  for (int g = 0; g < MAXG; ++g) {
+    const float o = __shfl_xor_sync(0xffffffffu, s[g], 1);
+    const float tot = hf == 0 ? s[g] + o : o + s[g];
+    if (g < G && hf == 0) ws[g * SLICE + sl] = p >= 0 ? tot : -INFINITY;
+  }
   __syncthreads();
   // per head: maximum and sum of exp(s - m) over the slice
   const int warp = th >> 5, lane = th & 31;
@@ -157,23 +168,52 @@ constexpr int sparse_attn_smem() {
          sa::SLICE * 4 + 2 * sa::MAXG * 4;
 }
 
+// The slices' maxima and sums of one (query, head) are staged in shared
+// memory first (all loads issued before any is used), then every thread forms
+// the weights exp(m_s - M) and adds its feature over the slices, eight
+// loads in flight at a time.
 template <int D>
 __global__ void __launch_bounds__(D)
     sparse_attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                int nsplit, uint16_t* __restrict__ out) {
+  __shared__ float f_s[sa::MAXSPLIT], l_s[sa::MAXSPLIT];
+  __shared__ float red[D / 32];
   const int th = threadIdx.x;
   const size_t th_h = blockIdx.x;            // t * Hq + h
+  float m_loc = -INFINITY;
+  for (int s = th; s < nsplit; s += D) {
+    const float2 ml = *reinterpret_cast<const float2*>(part_ml + (th_h * nsplit + s) * 2);
+    f_s[s] = ml.x;
+    l_s[s] = ml.y;
+    m_loc = fmaxf(m_loc, ml.x);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m_loc = fmaxf(m_loc, __shfl_xor_sync(0xffffffffu, m_loc, off));
+  if ((th & 31) == 0) red[th >> 5] = m_loc;
+  __syncthreads();
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part_ml[(th_h * nsplit + s) * 2]);
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
+  // weights of the slices (0 for a slice with no valid slot)
+  for (int s = th; s < nsplit; s += D)
+    f_s[s] = (M == -INFINITY || f_s[s] == -INFINITY) ? 0.f : __expf(f_s[s] - M);
+  __syncthreads();
   float num = 0.f, den = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float m = part_ml[(th_h * nsplit + s) * 2];
-      if (m == -INFINITY) continue;
-      const float f = __expf(m - M);
-      den = fmaf(f, part_ml[(th_h * nsplit + s) * 2 + 1], den);
-      num = fmaf(f, part_o[(th_h * nsplit + s) * D + th], num);
+  const float* po = part_o + th_h * nsplit * D + th;
+  int s = 0;
+  for (; s + 8 <= nsplit; s += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = po[(size_t)(s + u) * D];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      den = fmaf(f_s[s + u], l_s[s + u], den);
+      num = fmaf(f_s[s + u], v[u], num);
     }
+  }
+  for (; s < nsplit; ++s) {
+    den = fmaf(f_s[s], l_s[s], den);
+    num = fmaf(f_s[s], po[(size_t)s * D], num);
   }
   const float o = den > 0.f ? num / den : 0.f;
   out[th_h * D + th] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
