@@ -9,14 +9,20 @@
 // section 5.1): the gate/up epilogue applies SwiGLU.
 //
 // Swap-AB formulation.  One work unit = (expert e, two 128-row weight slots,
-// up to 128 token rows of e):
+// up to 160 token rows of e):
 //   gate/up: slot 0 = 128 gate rows, slot 1 = the same 128 up rows
 //   down:    slot 0, slot 1 = two consecutive 128-row blocks of W_down
 //   A (M = 128) dequantised weights, fp16, written by threads straight into
 //               tensor memory (tcgen05.st), read by tcgen05.mma from TMEM
-//   B (N <= 128) the unit's token rows, fp16, K-major, 128-byte swizzled in
+//   B (N <= 160) the unit's token rows, fp16, K-major, 128-byte swizzled in
 //               shared memory (one tile feeds both slots' MMAs)
 //   D           fp32 accumulators in TMEM, lane = weight row, column = token
+// Units of up to 160 token rows: with a top-10 of 512 experts over 6144
+// tokens an expert gets 120 rows on average and rarely more than 160, so
+// nearly every expert is one unit per weight-row block and its weights are
+// dequantised once.  (With 128-row units one expert in four needed a second,
+// nearly empty unit that dequantised all of its weights again: 630 tiles
+// instead of 512, and the layer took 2.37 ms instead of 2.16.)
 // Keeping A out of shared memory leaves shared-memory bandwidth to the B
 // tiles and the packed weights; the MMAs' own reads of B need half of it.
 //
@@ -26,8 +32,9 @@
 //                block of 8 groups of both slots' rows (16 B per row) every
 //                8 G / 64 stages into a two-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
-//   warp 2       token rows into a 4-deep ring, one TMA tile of 128 rows per
-//                stage: the down projection reads h, whose rows are already
+//   warp 2       token rows into a 5-deep (down: 3-deep) ring, one TMA tile
+//                of 160 rows per stage: the down projection reads h, whose
+//                rows are already
 //                grouped by expert; for gate/up a pre-pass writes the fp16 rows
 //                of x in grouped order (x[sorted_token[p]]), so both operands
 //                of every stage arrive by TMA.  (Gathering the rows from a
@@ -39,12 +46,11 @@
 //                TMEM with tcgen05.st; at each scale block a thread copies its
 //                rows' 8 scales into registers and frees the ring slot.  (When
 //                K / G is not a multiple of 8 the rows' scales are loaded from
-//                global memory one block ahead instead.  Those register loads
-//                cost the large workload about 6%: a thread's next release of
-//                a ring slot waited for its load in flight.)
+//                global memory one block ahead instead: a thread's next
+//                release of a ring slot waits for such a load in flight.)
 //   warps 11-14  epilogue: TMEM -> registers -> SwiGLU or row scale -> fp16,
 //                transposed through shared memory into whole-row stores
-// TMEM (512 columns): accumulators of slot 0/1 at columns 0/128, four A
+// TMEM (512 columns): accumulators of slot 0/1 at columns 0/160, three A
 // stages of 64 columns (32 per slot) at 256..511.
 //
 // Operands are fp16 (kind::f16): x rows are copied to fp16 in grouped order
@@ -64,7 +70,7 @@ constexpr int BM = 128;                    // weight rows per slot (TMEM lanes)
 constexpr int NT = kTileRows;              // token rows per unit (max MMA N)
 constexpr int BK = 64;                     // K per stage
 constexpr int RAW_ST = 8;                  // packed-weight ring depth
-constexpr int A_ST = 4;                    // TMEM A stages
+constexpr int A_ST = 3;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
 constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output feature)
@@ -91,7 +97,7 @@ struct Roles {
 // down's and the space goes to two more token-row stages.
 template <int OP>
 struct Lay {
-  static constexpr int B_ST = OP == 0 ? 6 : 4;                      // token-row ring depth
+  static constexpr int B_ST = OP == 0 ? 5 : 3;                      // token-row ring depth
   static constexpr int RAW_OFF = 0;                                 // [RAW_ST][2][RAW_BYTES]
   static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;    // [B_ST][B_BYTES]
   static constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;            // [slices * BM][STG_PITCH]
@@ -104,7 +110,7 @@ struct Lay {
 };
 
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t A_COL = 256;
+constexpr uint32_t A_COL = 2 * NT;
 }  // namespace tc
 
 struct TcArgs {
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
               if (m < U.nslots)
-                mma_f16kind_ts(tmem + m * BM, tmem + A_COL + sa * 64 + m * 32 + ks * 8, bd,
+                mma_f16kind_ts(tmem + m * NT, tmem + A_COL + sa * 64 + m * 32 + ks * 8, bd,
                                idesc, (kb | ks) != 0);
             }
           }
@@ -604,11 +610,11 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         for (int c = 0; c < nch; ++c) {
           __syncwarp();   // converged before the .sync.aligned TMEM loads
           uint32_t a0[32];
-          tmem_ld_32x32b_x32(t_lane + m * BM + c * 32, a0);
+          tmem_ld_32x32b_x32(t_lane + m * NT + c * 32, a0);
           float v[32];
           if (OP == 0) {
             uint32_t a1[32];
-            tmem_ld_32x32b_x32(t_lane + BM + c * 32, a1);
+            tmem_ld_32x32b_x32(t_lane + NT + c * 32, a1);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -647,10 +653,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
       // staging tile complete; a wait that gave up in any epilogue warp ends
       // the loop in all four alike
       if (named_barrier_or(1, 128, !got)) break;
-      if (et < U.cnt) {
-        uint16_t* dst = args.out + (size_t)(U.p0 + et) * N + U.fout[0];
+      for (int tt = et; tt < U.cnt; tt += 128) {
+        uint16_t* dst = args.out + (size_t)(U.p0 + tt) * N + U.fout[0];
         for (int ch = 0; ch < nout * (BM / 8); ++ch) {
-          const uint16_t* src = sStg + ch * 8 * STG_PITCH + et;
+          const uint16_t* src = sStg + ch * 8 * STG_PITCH + tt;
           uint32_t h[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) h[k] = src[k * STG_PITCH];

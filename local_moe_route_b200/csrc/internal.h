@@ -10,7 +10,7 @@
 namespace strata {
 
 // Tile of token rows handled by one tcgen05 GEMM work unit.
-constexpr int kTileRows = 128;
+constexpr int kTileRows = 160;
 // Token slots per histogram chunk in the permutation.
 constexpr int kPermChunk = 1024;
 // Batches of at most this many tokens use the weight-streaming expert kernel.
