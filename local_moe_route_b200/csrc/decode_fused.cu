@@ -292,15 +292,16 @@ __device__ __forceinline__ float df_key_value(uint32_t k) {
 
 // Top k of token t by one warp: lane l holds experts l, l + 32, ... (NV per
 // lane, E <= 32 NV) as order-preserving keys (NaN as -inf, -0 as +0; absent
-// and taken entries as 0, below every key).  Each round every lane offers
+// entries as 0, below every key).  Each round every lane offers
 // its best entry (largest key, then lowest index), the warp takes the
 // largest key and, among the lanes offering it, the lowest expert index (two
-// warp reductions), and the owning lane clears that entry: exact ties go to
-// the lower expert index and NaN never wins.  Then the softmax over the k.
+// warp reductions), and the owning lane marks that entry taken: exact ties go
+// to the lower expert index and NaN never wins.  Then the softmax over the k.
 template <int NV>
 __device__ __forceinline__ void df_topk(const FusedArgs& a, const Route& R, const float* logit_s,
                                         int t, int lane) {
   uint32_t key[NV];
+  uint32_t taken = 0;                         // entries already picked
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int e = lane + 32 * i;
@@ -315,7 +316,7 @@ __device__ __forceinline__ void df_topk(const FusedArgs& a, const Route& R, cons
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = i & 3;
-      if (key[i] > bk[c]) {                 // the first of equal keys stays (lower index)
+      if (!((taken >> i) & 1u) && key[i] > bk[c]) {                 // the first of equal keys stays (lower index)
         bk[c] = key[i];
         bs[c] = i;
       }
@@ -329,11 +330,7 @@ __device__ __forceinline__ void df_topk(const FusedArgs& a, const Route& R, cons
     }
     const uint32_t wk = __reduce_max_sync(0xffffffffu, bk[0]);
     const int wi = __reduce_min_sync(0xffffffffu, bk[0] == wk ? lane + 32 * bs[0] : 0x7fffffff);
-    if ((wi & 31) == lane) {
-#pragma unroll
-      for (int i = 0; i < NV; ++i)
-        if (i == (wi >> 5)) key[i] = 0u;
-    }
+    if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
     if (j == 0) top = wk;
     if (lane == j) {
       my_key = wk;

@@ -178,22 +178,31 @@ __global__ void __launch_bounds__(256)
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * d);
-#pragma unroll 2
-    for (int c = lane; c < cpr; c += 32) {
-      const uint4 v = __ldg(src + c);
-      float e[8];
-      e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
-      e[4] = bf16_lo(v.z); e[5] = bf16_hi(v.z); e[6] = bf16_lo(v.w); e[7] = bf16_hi(v.w);
+    // four 16-byte loads of the row in flight per lane before any is used;
+    // the copy is written once and read back once by the GEMM's TMA, so it
+    // goes out with an evict-first hint
+    for (int c0 = lane; c0 < cpr; c0 += 4 * 32) {
+      uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
-      // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
-      // weight dequantisation produces)
-      uint4 o;
-      o.x = pack_f16x2(e[0], e[4]);
-      o.y = pack_f16x2(e[1], e[5]);
-      o.z = pack_f16x2(e[2], e[6]);
-      o.w = pack_f16x2(e[3], e[7]);
-      dst[c] = o;
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < cpr) v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c0 + 32 * u >= cpr) break;
+        float e[8];
+        e[0] = bf16_lo(v[u].x); e[1] = bf16_hi(v[u].x); e[2] = bf16_lo(v[u].y); e[3] = bf16_hi(v[u].y);
+        e[4] = bf16_lo(v[u].z); e[5] = bf16_hi(v[u].z); e[6] = bf16_lo(v[u].w); e[7] = bf16_hi(v[u].w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) over |= fabsf(e[j]) > 65504.f;
+        // K order within the group of 8: 0, 4, 1, 5, 2, 6, 3, 7 (the order the
+        // weight dequantisation produces)
+        uint4 o;
+        o.x = pack_f16x2(e[0], e[4]);
+        o.y = pack_f16x2(e[1], e[5]);
+        o.z = pack_f16x2(e[2], e[6]);
+        o.w = pack_f16x2(e[3], e[7]);
+        __stcs(dst + c0 + 32 * u, o);
+      }
     }
   }
   if (over) atomicOr(err, kErrRange);

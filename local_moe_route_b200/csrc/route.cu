@@ -283,9 +283,25 @@ cudaError_t launch_router_logits_simt(const uint16_t* x, const uint16_t* w_route
 }
 
 // ===========================================================================
-// Top-k + softmax, one warp per token.  Lane l holds experts l, l+32, ...
-// Each of the k rounds takes the warp-wide maximum (ties: lower index),
-// marks it taken, and lane j keeps the j-th pick.
+// Order-preserving 32-bit key of a logit: larger float, larger key; NaN maps
+// to the key of -inf and -0 to that of +0, so keys compare as the selection
+// treats the floats.  Key 0 lies below every key (absent / taken entries).
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  if (f != f) f = -INFINITY;
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Top-k + softmax, one warp per token.  Lane l holds experts l, l+32, ... as
+// keys.  Each of the k rounds: every lane offers its best entry (largest key,
+// lowest index among equal keys), the warp takes the largest key and the
+// lowest expert index offering it (two redux.sync reductions), and the owning
+// lane marks that entry taken; lane j keeps the j-th pick.  Exact ties go to the
+// lower expert index and NaN never wins.
 template <int VPL>
 __global__ void __launch_bounds__(128)
     topk_softmax_kernel(const float* __restrict__ partial, int ksplit,
@@ -295,55 +311,51 @@ __global__ void __launch_bounds__(128)
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (t >= T) return;
-  float v[VPL];
-  uint32_t taken = 0;
+  uint32_t key[VPL];
+  uint32_t taken = 0;                         // entries already picked
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
+    key[i] = 0u;
     if (e < E) {
       float acc = 0.f;
       for (int sp = 0; sp < ksplit; ++sp) acc += partial[((size_t)sp * T + t) * E + e];
       if (bias) acc += bias[e];
       if (logits_out) logits_out[(size_t)t * E + e] = acc;
-      v[i] = acc;
-    } else {
-      v[i] = -INFINITY;
-      taken |= 1u << i;
+      key[i] = logit_key(acc);
     }
   }
-  float my_v = 0.f, top = 0.f;
+  uint32_t my_key = 0, top = 0;
   int my_i = 0;
   for (int j = 0; j < k; ++j) {
-    float best = -INFINITY;
-    int bi = 0x7fffffff;
+    // up to four independent chains over i mod 4, merged in index order
+    uint32_t bk[4] = {0u, 0u, 0u, 0u};
+    int bs[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      if (!((taken >> i) & 1u)) {
-        const float c = (v[i] != v[i]) ? -INFINITY : v[i];   // NaN never wins
-        const int e = lane + 32 * i;
-        if (c > best || (c == best && e < bi)) {
-          best = c;
-          bi = e;
-        }
+      const int c = i & 3;
+      if (!((taken >> i) & 1u) && key[i] > bk[c]) {                   // the first of equal keys stays (lower index)
+        bk[c] = key[i];
+        bs[c] = i;
       }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (ob > best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
+    for (int c = 1; c < 4; ++c) {
+      if (bk[c] > bk[0] || (bk[c] == bk[0] && bs[c] < bs[0])) {
+        bk[0] = bk[c];
+        bs[0] = bs[c];
       }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (j == 0) top = best;
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk[0]);
+    const int wi = __reduce_min_sync(0xffffffffu, bk[0] == wk ? lane + 32 * bs[0] : 0x7fffffff);
+    if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
+    if (j == 0) top = wk;
     if (lane == j) {
-      my_v = best;
-      my_i = bi;
+      my_key = wk;
+      my_i = wi;
     }
   }
-  const float ex = (lane < k) ? expf(my_v - top) : 0.f;
+  const float ex = (lane < k) ? expf(key_logit(my_key) - key_logit(top)) : 0.f;
   float sum = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);

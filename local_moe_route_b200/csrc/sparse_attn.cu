@@ -53,22 +53,37 @@ __global__ void __launch_bounds__(sa::THREADS)
   float* mx = reinterpret_cast<float*>(rows + SLICE);              // [MAXG]
   float* sm = mx + MAXG;                                           // [MAXG]
   const int th = threadIdx.x;
+  // the slice's index slots and the G query rows of this KV head: every load
+  // issued before the first barrier (16-byte loads of q, at most two per
+  // thread: G * D <= 16 * 128)
+  int p = -1;
+  const int slot = split * SLICE + th;
+  if (th < SLICE && slot < P) p = idx[(size_t)t * P + slot];
+  uint4 qv[2];
+  const uint16_t* qrow = q + ((size_t)t * Hq + hk * G) * D;   // G rows of D, contiguous
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = (th + u * THREADS) * 8;
+    if (i < G * D) qv[u] = *reinterpret_cast<const uint4*>(qrow + i);
+  }
   if (th < SLICE) {
-    const int slot = split * SLICE + th;
-    int p = -1;
-    if (slot < P) {
-      p = idx[(size_t)t * P + slot];
-      if (p >= L) {
-        atomicOr(err, kErrIndex);
-        p = -1;
-      }
+    if (p >= L) {
+      atomicOr(err, kErrIndex);
+      p = -1;
     }
     rows[th] = p;
   }
-  for (int i = th; i < G * D; i += THREADS) {
-    const int g = i / D, dd = i % D;
-    qs[g * D + dd] =
-        __uint_as_float((uint32_t)q[((size_t)t * Hq + hk * G + g) * D + dd] << 16) * scale;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = (th + u * THREADS) * 8;
+    if (i < G * D) {
+      const uint4 v = qv[u];
+      float* dst = qs + i;                   // [g][dd] with g * D + dd = i
+      dst[0] = bf16_lo(v.x) * scale; dst[1] = bf16_hi(v.x) * scale;
+      dst[2] = bf16_lo(v.y) * scale; dst[3] = bf16_hi(v.y) * scale;
+      dst[4] = bf16_lo(v.z) * scale; dst[5] = bf16_hi(v.z) * scale;
+      dst[6] = bf16_lo(v.w) * scale; dst[7] = bf16_hi(v.w) * scale;
+    }
   }
   __syncthreads();
   // the slice's K and V rows into shared memory: every copy issued before
@@ -89,11 +104,11 @@ __global__ void __launch_bounds__(sa::THREADS)
   // scores of slot th / 2 for the G heads: the two threads of a slot take
   // one half of D each and add their sums (fixed order: lower half first)
   const int sl = th >> 1, hf = th & 1;
-  const int p = rows[sl];
+  const int pr_s = rows[sl];
   float s[MAXG];
 #pragma unroll
   for (int g = 0; g < MAXG; ++g) s[g] = 0.f;
-  if (p >= 0) {
+  if (pr_s >= 0) {
     const uint4* kr = reinterpret_cast<const uint4*>(ks + sl * RP) + hf * (CPR / 2);
 #pragma unroll 4
     for (int c = 0; c < CPR / 2; ++c) {
@@ -114,7 +129,7 @@ __global__ void __launch_bounds__(sa::THREADS)
   for (int g = 0; g < MAXG; ++g) {
     const float o = __shfl_xor_sync(0xffffffffu, s[g], 1);
     const float tot = hf == 0 ? s[g] + o : o + s[g];
-    if (g < G && hf == 0) ws[g * SLICE + sl] = p >= 0 ? tot : -INFINITY;
+    if (g < G && hf == 0) ws[g * SLICE + sl] = pr_s >= 0 ? tot : -INFINITY;
   }
   __syncthreads();
   // per head: maximum and sum of exp(s - m) over the slice
