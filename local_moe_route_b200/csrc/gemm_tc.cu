@@ -28,11 +28,11 @@
 //
 // Warp roles (480 threads, persistent, one CTA per SM):
 //   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
-//                swizzle) into an 8-deep ring, and of the group scales: one
-//                block of 8 groups of both slots' rows (16 B per row) every
-//                8 G / 64 stages into a two-deep ring
+//                swizzle) into an 8-deep (down: 5-deep) ring, and of the
+//                group scales: one block of 8 groups of both slots' rows
+//                (16 B per row) every 8 G / 64 stages into a two-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
-//   warp 2       token rows into a 5-deep (down: 3-deep) ring, one TMA tile
+//   warp 2       token rows into a 5-deep (down: 4-deep) ring, one TMA tile
 //                of 160 rows per stage: the down projection reads h, whose
 //                rows are already
 //                grouped by expert; for gate/up a pre-pass writes the fp16 rows
@@ -69,7 +69,6 @@ namespace tc {
 constexpr int BM = 128;                    // weight rows per slot (TMEM lanes)
 constexpr int NT = kTileRows;              // token rows per unit (max MMA N)
 constexpr int BK = 64;                     // K per stage
-constexpr int RAW_ST = 8;                  // packed-weight ring depth
 constexpr int A_ST = 3;                    // TMEM A stages
 constexpr int RAW_BYTES = BM * BK / 2;     // 4 KB per slot
 constexpr int B_BYTES = NT * BK * 2;       // 16 KB
@@ -97,7 +96,8 @@ struct Roles {
 // down's and the space goes to two more token-row stages.
 template <int OP>
 struct Lay {
-  static constexpr int B_ST = OP == 0 ? 5 : 3;                      // token-row ring depth
+  static constexpr int B_ST = OP == 0 ? 5 : 4;                      // token-row ring depth
+  static constexpr int RAW_ST = OP == 0 ? 8 : 5;                    // packed-weight ring depth
   static constexpr int RAW_OFF = 0;                                 // [RAW_ST][2][RAW_BYTES]
   static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;    // [B_ST][B_BYTES]
   static constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;            // [slices * BM][STG_PITCH]
@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   using namespace tc;
   using Ly = Lay<OP>;
   constexpr int B_ST = Ly::B_ST;
+  constexpr int RAW_ST = Ly::RAW_ST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
