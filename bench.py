@@ -50,6 +50,7 @@ METRIC = "MoE-layer tokens/s at T=6144, 512 experts top-10; % of tensor/HBM roof
 # profiles/traffic.json stand only while these files are unchanged.
 KERNEL_SOURCES = {
     "gemm_gate_up_large": ["local_moe_route_b200/csrc/gemm_tc.cu",
+                           "local_moe_route_b200/csrc/dequant.cuh",
                            "local_moe_route_b200/csrc/common.cuh"],
     "gemm_gate_up_verify4": ["local_moe_route_b200/csrc/gemm_decode.cu",
                              "local_moe_route_b200/csrc/common.cuh"],
@@ -516,7 +517,7 @@ def run_ours(args, wl):
 
 def gate_up_kernels(T):
     if T > 8:
-        return ("work lists + grouped fp16 copy of x + moe_gemm_q4_tc_kernel<0,0> "
+        return ("work lists + grouped fp16 copy of x + moe_gemm_q4_tc_kernel<0,0,1> "
                 "(gate/up + SwiGLU), one entry-point call")
     return "work lists + moe_gemm_q4_decode_kernel<2, G> (gate/up + SwiGLU), one entry-point call"
 
