@@ -609,6 +609,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     const int et = threadIdx.x - Roles<OP>::W_EPI * 32;   // 0..127
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     bool ov = false;            // an output of this thread overflowed fp16
+    __half2 omax = __float2half2_rn(0.f);   // largest |output| of the current unit
     for (int i = 0; i < my_units; ++i) {
       const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
       const bool got = mbar_wait_warp(acc_full, i & 1, abort_flag, args.err);
@@ -643,46 +644,67 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
               }
             }
           }
-          // columns past the unit's rows hold no result of this unit
+          // columns past the unit's rows hold no result of this unit; the
+          // others are checked for fp16 overflow on the packed pairs (a
+          // running maximum of |h| that lets NaN through, tested per unit)
           const int lim = U.cnt - c * 32;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ov |= j < lim && f16_overflows(v[j]);
-#pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
-            uint4 o;
-            o.x = pack_f16x2(v[8 * k4 + 0], v[8 * k4 + 1]);
-            o.y = pack_f16x2(v[8 * k4 + 2], v[8 * k4 + 3]);
-            o.z = pack_f16x2(v[8 * k4 + 4], v[8 * k4 + 5]);
-            o.w = pack_f16x2(v[8 * k4 + 6], v[8 * k4 + 7]);
-            *reinterpret_cast<uint4*>(frow + c * 32 + 8 * k4) = o;
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              o[u] = pack_f16x2(v[8 * k4 + 2 * u], v[8 * k4 + 2 * u + 1]);
+              const int j = 8 * k4 + 2 * u;
+              const uint32_t live = j + 1 < lim ? o[u] : (j < lim ? (o[u] & 0xFFFFu) : 0u);
+              omax = __hmax2_nan(omax, __habs2(*reinterpret_cast<const __half2*>(&live)));
+            }
+            *reinterpret_cast<uint4*>(frow + c * 32 + 8 * k4) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
       }
       tc_fence_before();
       if (got) mbar_arrive(acc_empty);
+      {
+        // an overflowed (or NaN) half has all exponent bits set
+        const uint32_t mb = *reinterpret_cast<const uint32_t*>(&omax);
+        ov |= (mb & 0x7C00u) == 0x7C00u || (mb & 0x7C000000u) == 0x7C000000u;
+        omax = __float2half2_rn(0.f);
+      }
       // staging tile complete; a wait that gave up in any epilogue warp ends
       // the loop in all four alike
       if (named_barrier_or(1, 128, !got)) break;
-      for (int tt = et; tt < U.cnt; tt += 128) {
-        uint16_t* dst = args.out + (size_t)(U.p0 + tt) * N + U.fout[0];
-        for (int ch = 0; ch < nout * (BM / 8); ++ch) {
-          const uint16_t* src = sStg + ch * 8 * STG_PITCH + tt;
-          uint32_t h[8];
+      // copy-out: item = (4 consecutive tokens, 8 consecutive features);
+      // eight 8-byte loads give the 4 x 8 block, four 16-byte stores write it
+      const int ntg = (U.cnt + 3) >> 2;
+      const int items = ntg * nout * (BM / 8);
+      for (int it = et; it < items; it += 128) {
+        const int tg = it % ntg, ch = it / ntg;
+        const uint16_t* src = sStg + ch * 8 * STG_PITCH + 4 * tg;
+        uint2 h[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) h[k] = src[k * STG_PITCH];
+        for (int k = 0; k < 8; ++k) h[k] = *reinterpret_cast<const uint2*>(src + k * STG_PITCH);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tt = 4 * tg + u;
+          if (tt >= U.cnt) break;
+          // token u's value of feature k: half (u & 1) of h[k].x (u < 2) or h[k].y
+          uint32_t f[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) f[k] = u < 2 ? h[k].x : h[k].y;
+          const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;
           uint4 o;
           if (OP == 0 && ILV) {      // features 0,4 | 1,5 | 2,6 | 3,7 (see GemmProblem)
-            o.x = __byte_perm(h[0], h[4], 0x5410);
-            o.y = __byte_perm(h[1], h[5], 0x5410);
-            o.z = __byte_perm(h[2], h[6], 0x5410);
-            o.w = __byte_perm(h[3], h[7], 0x5410);
+            o.x = __byte_perm(f[0], f[4], sel);
+            o.y = __byte_perm(f[1], f[5], sel);
+            o.z = __byte_perm(f[2], f[6], sel);
+            o.w = __byte_perm(f[3], f[7], sel);
           } else {
-            o.x = __byte_perm(h[0], h[1], 0x5410);
-            o.y = __byte_perm(h[2], h[3], 0x5410);
-            o.z = __byte_perm(h[4], h[5], 0x5410);
-            o.w = __byte_perm(h[6], h[7], 0x5410);
+            o.x = __byte_perm(f[0], f[1], sel);
+            o.y = __byte_perm(f[2], f[3], sel);
+            o.z = __byte_perm(f[4], f[5], sel);
+            o.w = __byte_perm(f[6], f[7], sel);
           }
-          *reinterpret_cast<uint4*>(dst + ch * 8) = o;
+          *reinterpret_cast<uint4*>(args.out + (size_t)(U.p0 + tt) * N + U.fout[0] + ch * 8) = o;
         }
       }
       named_barrier_sync(1, 128);                     // staging tile free again
