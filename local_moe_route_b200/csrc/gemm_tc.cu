@@ -26,11 +26,13 @@
 // Keeping A out of shared memory leaves shared-memory bandwidth to the B
 // tiles and the packed weights; the MMAs' own reads of B need half of it.
 //
-// Warp roles (480 threads, persistent, one CTA per SM):
-//   warp 0       TMA of packed int4 rows (32 B per row per 64-K stage, 32-byte
-//                swizzle) into an 8-deep (down: 5-deep) ring, and of the
-//                group scales: one block of 8 groups of both slots' rows
-//                (16 B per row) every 8 G / 64 stages into a two-deep ring
+// Warp roles (gate/up 480 threads, down 736; persistent, one CTA per SM):
+//   warp 0       TMA of packed int4 rows into a ring of 8 (down: 6) K stages
+//                of 64: one copy covers two K stages when K is a multiple of
+//                128 (a 64-byte row segment per weight row, 64-byte swizzle;
+//                otherwise 32 bytes, 32-byte swizzle), and of the group
+//                scales: one block of 8 groups of both slots' rows (16 B per
+//                row) every 8 G / 64 stages into a two-deep ring
 //   warp 1       tcgen05.mma issue (one thread)
 //   warp 2       token rows into a 5-deep (down: 4-deep) ring, one TMA tile
 //                of 160 rows per stage: the down projection reads h, whose
@@ -41,17 +43,18 @@
 //                token-order copy with tile::gather4 copies instead, 32 per
 //                stage, left the MMA waiting on them 64% of the time and
 //                doubled the kernel's time at T = 6144.)
-//   warps 3-10   two (down: three) dequantising warpgroups taking the
-//                stages round-robin; thread = weight row; fp16 pairs go to
+//   warps 3-10   two (down: three, warps 3-14) dequantising warpgroups taking
+//                the stages round-robin; thread = weight row; fp16 pairs go to
 //                TMEM with tcgen05.st; at each scale block a thread copies its
 //                rows' 8 scales into registers and frees the ring slot.  (When
 //                K / G is not a multiple of 8 the rows' scales are loaded from
 //                global memory one block ahead instead: a thread's next
 //                release of a ring slot waits for such a load in flight.)
-//   warps 11-14  epilogue: TMEM -> registers -> SwiGLU or row scale -> fp16,
+//   warps 11-14  epilogue (down: warps 15-22, four per 128-feature slice):
+//                TMEM -> registers -> SwiGLU or row scale -> fp16,
 //                transposed through shared memory into whole-row stores
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/160, three A
-// stages of 64 columns (32 per slot) at 256..511.
+// stages of 64 columns (32 per slot) at 320..511.
 //
 // Operands are fp16 (kind::f16): x rows are copied to fp16 in grouped order
 // once per call (exact for |x| < 65504), h is kept in fp16, and each weight is RNE_fp16(q * s): fp16
@@ -88,18 +91,25 @@ template <int OP>
 struct Roles {
   static constexpr int NWG = OP == 0 ? 2 : 3;
   static constexpr int W_EPI = W_DQ + 4 * NWG;
-  static constexpr int THREADS = (W_EPI + 4) * 32;
+  // epilogue warps: down has two 128-feature slices per unit and gives each
+  // its own four warps, so the accumulator is read out in half the time
+  static constexpr int NEPI = OP == 0 ? 4 : 8;
+  static constexpr int THREADS = (W_EPI + NEPI) * 32;
 };
 
 // Shared memory per operation: gate/up writes one 128-feature slice per unit
 // (SwiGLU merges the two slots), so its staging tile is half the size of
 // down's and the space goes to two more token-row stages.
-template <int OP>
+// RK: K stages per packed-weight copy (2 when K is a multiple of 128: one
+// 64-byte row segment per weight row and copy instead of two 32-byte ones).
+template <int OP, int RK>
 struct Lay {
   static constexpr int B_ST = OP == 0 ? 5 : 4;                      // token-row ring depth
-  static constexpr int RAW_ST = OP == 0 ? 8 : 5;                    // packed-weight ring depth
-  static constexpr int RAW_OFF = 0;                                 // [RAW_ST][2][RAW_BYTES]
-  static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_BYTES;    // [B_ST][B_BYTES]
+  // packed-weight ring depth in copies (8 / 5 K stages of 64, rounded up)
+  static constexpr int RAW_ST = OP == 0 ? 8 / RK : (RK == 1 ? 5 : 3);
+  static constexpr int RAW_SLOT = RK * RAW_BYTES;                   // one slot of one copy
+  static constexpr int RAW_OFF = 0;                                 // [RAW_ST][2][RAW_SLOT]
+  static constexpr int B_OFF = RAW_OFF + RAW_ST * 2 * RAW_SLOT;     // [B_ST][B_BYTES]
   static constexpr int STG_OFF = B_OFF + B_ST * B_BYTES;            // [slices * BM][STG_PITCH]
   static constexpr int STG_BYTES = (OP == 0 ? 1 : 2) * BM * STG_PITCH * 2;
   static constexpr int SC_OFF = STG_OFF + STG_BYTES;                 // [2][2][BM][8] fp16
@@ -107,7 +117,13 @@ struct Lay {
   static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = 1024 + MISC_OFF + 64;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
 };
+
+// Packed-weight copies of RK K stages when the group scales come by TMA
+// (K / G a multiple of 8 implies K a multiple of 128 for G >= 16).
+template <bool STMA>
+__host__ __device__ constexpr int raw_k_stages() { return STMA ? 2 : 1; }
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t A_COL = 2 * NT;
@@ -226,9 +242,11 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
                           const __grid_constant__ CUtensorMap map_s0,
                           const __grid_constant__ CUtensorMap map_s1, const TcArgs args) {
   using namespace tc;
-  using Ly = Lay<OP>;
+  constexpr int RK = raw_k_stages<STMA>();
+  using Ly = Lay<OP, RK>;
   constexpr int B_ST = Ly::B_ST;
   constexpr int RAW_ST = Ly::RAW_ST;
+  constexpr int RAW_SLOT = Ly::RAW_SLOT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -259,7 +277,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < RAW_ST; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], BM);
+      mbar_init(&raw_empty[s], RK * BM);   // every K stage of the copy, one warpgroup each
     }
     for (int s = 0; s < B_ST; ++s) {
       mbar_init(&b_full[s], 1);
@@ -270,7 +288,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, BM);
+    mbar_init(acc_empty, Roles<OP>::NEPI * 32);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sc_full[b], 1);
       mbar_init(&sc_empty[b], Roles<OP>::NWG * BM);
@@ -324,16 +342,18 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
                         &sc_full[ss]);
             ++gs;
           }
-          const int s = g % RAW_ST;
-          if (g >= (uint32_t)RAW_ST &&
-              !mbar_wait(&raw_empty[s], ((g / RAW_ST) - 1) & 1, abort_flag, args.err)) {
+          if (kb % RK != 0) continue;       // this copy holds RK K stages
+          const uint32_t gr = g / RK;
+          const int s = gr % RAW_ST;
+          if (gr >= (uint32_t)RAW_ST &&
+              !mbar_wait(&raw_empty[s], ((gr / RAW_ST) - 1) & 1, abort_flag, args.err)) {
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&raw_full[s], 2 * RAW_BYTES);
-          tma_load_2d(sRaw + (s * 2 + 0) * RAW_BYTES, &map_q0, kb * (BK / 2), U.wrow[0],
+          mbar_arrive_expect_tx(&raw_full[s], 2 * RAW_SLOT);
+          tma_load_2d(sRaw + (s * 2 + 0) * RAW_SLOT, &map_q0, kb * (BK / 2), U.wrow[0],
                       &raw_full[s]);
-          tma_load_2d(sRaw + (s * 2 + 1) * RAW_BYTES, map_slot1, kb * (BK / 2), U.wrow[1],
+          tma_load_2d(sRaw + (s * 2 + 1) * RAW_SLOT, map_slot1, kb * (BK / 2), U.wrow[1],
                       &raw_full[s]);
         }
       }
@@ -534,16 +554,19 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         kb -= KB;
         ++iu;
       }
-      const int sr = g % RAW_ST, sa = g % A_ST;
-      if (!mbar_wait(&raw_full[sr], (g / RAW_ST) & 1, abort_flag, args.err)) break;
-      // packed words of this row; 32-byte swizzle puts chunk c at c ^ ((r >> 2) & 1)
+      const int sr = (g / RK) % RAW_ST, sa = g % A_ST;
+      if (!mbar_wait(&raw_full[sr], ((g / RK) / RAW_ST) & 1, abort_flag, args.err)) break;
+      // packed words of this row: 16-byte chunks 2j, 2j + 1 of the copy's row
+      // segment (j = the K stage within the copy); the 32-byte swizzle puts
+      // chunk c at c ^ ((r >> 2) & 1), the 64-byte one at c ^ ((r >> 1) & 3)
       uint4 raw[2][2];
-      const int sw = (r >> 2) & 1;
+      const int sw = RK == 1 ? (r >> 2) & 1 : (r >> 1) & 3;
+      const int c0 = 2 * (g % RK);
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
-        const uint8_t* rowp = sRaw + (sr * 2 + m) * RAW_BYTES + r * 32;
-        raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * sw);
-        raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * (sw ^ 1));
+        const uint8_t* rowp = sRaw + (sr * 2 + m) * RAW_SLOT + r * (RK * 32);
+        raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * (c0 ^ sw));
+        raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * ((c0 + 1) ^ sw));
       }
       // gate/up: both slots are dequantised into registers before this warp
       // waits for its A stage, so a stage the MMAs release is refilled at
@@ -605,8 +628,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     // after.  The transposition to the row-major output happens on the way
     // out: thread t gathers 8 features of token t and stores 16 bytes, while
     // the next unit's MMAs already run.
+    constexpr int ET = Roles<OP>::NEPI * 32;              // epilogue threads
     const int q = warp & 3;
-    const int et = threadIdx.x - Roles<OP>::W_EPI * 32;   // 0..127
+    const int et = threadIdx.x - Roles<OP>::W_EPI * 32;   // 0 .. ET - 1
+    const int esl = (warp - Roles<OP>::W_EPI) >> 2;       // the output slice this warp reads
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     bool ov = false;            // an output of this thread overflowed fp16
     __half2 omax = __float2half2_rn(0.f);   // largest |output| of the current unit
@@ -616,50 +641,76 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
       tc_fence_after();
       const int nch = (U.cnt + 31) >> 5;
       const int nout = OP == 0 ? 1 : U.nslots;        // 128-feature slices of output
-      for (int m = 0; m < nout && got; ++m) {
+      // 16 token values of slice m, columns 16 c16 .. -> fp16 pairs in the
+      // staging row of this thread's feature.  The pairs are checked for fp16
+      // overflow (a running maximum of |h| that lets NaN through, tested per
+      // unit); columns past the unit's rows hold no result of this unit, and
+      // only the last chunk of a unit can have such columns.
+      auto emit16 = [&](int m, int c16, const float* v) {
         uint16_t* frow = sStg + (m * BM + q * 32 + lane) * STG_PITCH;
-        for (int c = 0; c < nch; ++c) {
+        uint32_t o[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) o[u] = pack_f16x2(v[2 * u], v[2 * u + 1]);
+        const int lim = U.cnt - c16 * 16;
+        if (lim >= 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            omax = __hmax2_nan(omax, __habs2(*reinterpret_cast<const __half2*>(&o[u])));
+        } else {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 2 * u;
+            const uint32_t live = j + 1 < lim ? o[u] : (j < lim ? (o[u] & 0xFFFFu) : 0u);
+            omax = __hmax2_nan(omax, __habs2(*reinterpret_cast<const __half2*>(&live)));
+          }
+        }
+        *reinterpret_cast<uint4*>(frow + c16 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(frow + c16 * 16 + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+      };
+      if constexpr (OP == 0) {
+        for (int c = 0; c < nch && got; ++c) {
           __syncwarp();   // converged before the .sync.aligned TMEM loads
-          uint32_t a0[32];
-          tmem_ld_32x32b_x32(t_lane + m * NT + c * 32, a0);
+          uint32_t a0[32], a1[32];
+          tmem_ld_32x32b_x32(t_lane + c * 32, a0);
+          tmem_ld_32x32b_x32(t_lane + NT + c * 32, a1);
+          tmem_ld_wait_regs(a0);
+          tmem_ld_wait_regs(a1);
           float v[32];
-          if (OP == 0) {
-            uint32_t a1[32];
-            tmem_ld_32x32b_x32(t_lane + NT + c * 32, a1);
-            tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
+            v[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+          }
+          emit16(0, 2 * c, v);
+          emit16(0, 2 * c + 1, v + 16);
+        }
+      } else {
+        // the chunks of slice esl, one TMEM load and wait each (two loads
+        // per wait, or 16-column loads with the next one in flight, held the
+        // accumulator longer)
+        const int nq = got && esl < nout ? nch : 0;
+        auto taddr = [&](int c) { return t_lane + esl * NT + c * 32; };
+        auto convert = [&](int c, const uint32_t (&r)[32]) {
+          const int m = esl;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (args.row_scale) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float gv = __uint_as_float(a0[j]), uv = __uint_as_float(a1[j]);
-              v[j] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-            }
-          } else {
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a0[j]);
-            if (args.row_scale) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int t = c * 32 + j;
-                if (t < U.cnt) v[j] *= args.row_scale[U.p0 + t];
-              }
+              const int t = c * 32 + j;
+              if (t < U.cnt) v[j] *= args.row_scale[U.p0 + t];
             }
           }
-          // columns past the unit's rows hold no result of this unit; the
-          // others are checked for fp16 overflow on the packed pairs (a
-          // running maximum of |h| that lets NaN through, tested per unit)
-          const int lim = U.cnt - c * 32;
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            uint32_t o[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              o[u] = pack_f16x2(v[8 * k4 + 2 * u], v[8 * k4 + 2 * u + 1]);
-              const int j = 8 * k4 + 2 * u;
-              const uint32_t live = j + 1 < lim ? o[u] : (j < lim ? (o[u] & 0xFFFFu) : 0u);
-              omax = __hmax2_nan(omax, __habs2(*reinterpret_cast<const __half2*>(&live)));
-            }
-            *reinterpret_cast<uint4*>(frow + c * 32 + 8 * k4) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
+          emit16(m, 2 * c, v);
+          emit16(m, 2 * c + 1, v + 16);
+        };
+        for (int qq = 0; qq < nq; ++qq) {
+          __syncwarp();   // converged before the .sync.aligned TMEM loads
+          uint32_t ra[32];
+          tmem_ld_32x32b_x32(taddr(qq), ra);
+          tmem_ld_wait_regs(ra);
+          convert(qq, ra);
         }
       }
       tc_fence_before();
@@ -671,13 +722,13 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         omax = __float2half2_rn(0.f);
       }
       // staging tile complete; a wait that gave up in any epilogue warp ends
-      // the loop in all four alike
-      if (named_barrier_or(1, 128, !got)) break;
+      // the loop in all of them alike
+      if (named_barrier_or(1, ET, !got)) break;
       // copy-out: item = (4 consecutive tokens, 8 consecutive features);
       // eight 8-byte loads give the 4 x 8 block, four 16-byte stores write it
       const int ntg = (U.cnt + 3) >> 2;
       const int items = ntg * nout * (BM / 8);
-      for (int it = et; it < items; it += 128) {
+      for (int it = et; it < items; it += ET) {
         const int tg = it % ntg, ch = it / ntg;
         const uint16_t* src = sStg + ch * 8 * STG_PITCH + 4 * tg;
         uint2 h[8];
@@ -707,7 +758,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
           *reinterpret_cast<uint4*>(args.out + (size_t)(U.p0 + tt) * N + U.fout[0] + ch * 8) = o;
         }
       }
-      named_barrier_sync(1, 128);                     // staging tile free again
+      named_barrier_sync(1, ET);                      // staging tile free again
     }
     if (ov) atomicOr(args.err, kErrRange);
   }
@@ -724,8 +775,10 @@ template <int OP, bool ILV, bool STMA>
 static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cudaStream_t s) {
   CUtensorMap m0, m1;
   const uint64_t rows = (uint64_t)p.E * p.N;
+  constexpr int RK = tc::raw_k_stages<STMA>();
+  const CUtensorMapSwizzle raw_sw = RK == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (encode_tmap_2d(&m0, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q0, p.K / 2, rows, p.K / 2,
-                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
+                     RK * tc::BK / 2, tc::BM, raw_sw,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   m1 = m0;
@@ -738,7 +791,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
     return cudaErrorInvalidValue;
   if (OP == 0 &&
       encode_tmap_2d(&m1, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.q1, p.K / 2, rows, p.K / 2,
-                     tc::BK / 2, tc::BM, CU_TENSOR_MAP_SWIZZLE_32B,
+                     RK * tc::BK / 2, tc::BM, raw_sw,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // group scales [E * N][K / G] fp16, blocks of 8 groups x 128 rows
@@ -759,7 +812,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   {
     cudaError_t e = cudaFuncSetAttribute(moe_gemm_q4_tc_kernel<OP, ILV, STMA>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::Lay<OP>::SMEM);
+                                         tc::Lay<OP, RK>::SMEM);
     if (e != cudaSuccess) return e;
   }
   const int num_sms = sm_count();
@@ -789,7 +842,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const int FB = OP == 0 ? p.N / tc::BM : (p.N + 2 * tc::BM - 1) / (2 * tc::BM);
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-  moe_gemm_q4_tc_kernel<OP, ILV, STMA><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP>::SMEM, s>>>(
+  moe_gemm_q4_tc_kernel<OP, ILV, STMA><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP, RK>::SMEM, s>>>(
       m0, m1, mb, ms0, ms1, a);
   return cudaGetLastError();
 }
