@@ -26,14 +26,14 @@
 // Keeping A out of shared memory leaves shared-memory bandwidth to the B
 // tiles and the packed weights; the MMAs' own reads of B need half of it.
 //
-// Warp roles (gate/up 480 threads, down 736; persistent, one CTA per SM):
+// Warp roles (gate/up 512 threads, down 768; persistent, one CTA per SM):
 //   warp 0       TMA of packed int4 rows into a ring of 8 (down: 6) K stages
 //                of 64: one copy covers two K stages when K is a multiple of
 //                128 (a 64-byte row segment per weight row, 64-byte swizzle;
 //                otherwise 32 bytes, 32-byte swizzle), and of the group
 //                scales: one block of 8 groups of both slots' rows (16 B per
 //                row) every 8 G / 64 stages into a two-deep ring
-//   warp 1       tcgen05.mma issue (one thread)
+//   warps 1, 3   tcgen05.mma issue, one thread per slot
 //   warp 2       token rows into a 5-deep (down: 4-deep) ring, one TMA tile
 //                of 160 rows per stage: the down projection reads h, whose
 //                rows are already
@@ -43,14 +43,14 @@
 //                token-order copy with tile::gather4 copies instead, 32 per
 //                stage, left the MMA waiting on them 64% of the time and
 //                doubled the kernel's time at T = 6144.)
-//   warps 3-10   two (down: three, warps 3-14) dequantising warpgroups taking
+//   warps 4-11   two (down: three, warps 4-15) dequantising warpgroups taking
 //                the stages round-robin; thread = weight row; fp16 pairs go to
 //                TMEM with tcgen05.st; at each scale block a thread copies its
 //                rows' 8 scales into registers and frees the ring slot.  (When
 //                K / G is not a multiple of 8 the rows' scales are loaded from
 //                global memory one block ahead instead: a thread's next
 //                release of a ring slot waits for such a load in flight.)
-//   warps 11-14  epilogue (down: warps 15-22, four per 128-feature slice):
+//   warps 12-15  epilogue (down: warps 16-23, four per 128-feature slice):
 //                TMEM -> registers -> SwiGLU or row scale -> fp16,
 //                transposed through shared memory into whole-row stores
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/160, three A
@@ -81,7 +81,7 @@ constexpr int STG_PITCH = NT + 8;          // halves per staging row (one output
 constexpr int SC_GROUPS = 8;
 constexpr int SC_BYTES = 2 * BM * SC_GROUPS * 2;   // 4 KB per block
 
-constexpr int W_TMA = 0, W_MMA = 1, W_BTMA = 2, W_DQ = 3;
+constexpr int W_TMA = 0, W_MMA = 1, W_BTMA = 2, W_MMA2 = 3, W_DQ = 4;
 // Dequantising warpgroups take the stages round-robin: two for gate/up,
 // three for down, whose units are short (K = n) and leave the MMA warp
 // waiting on dequantisation more often (measured: down 0.73 -> 0.67 ms at the
@@ -114,7 +114,7 @@ struct Lay {
   static constexpr int STG_BYTES = (OP == 0 ? 1 : 2) * BM * STG_PITCH * 2;
   static constexpr int SC_OFF = STG_OFF + STG_BYTES;                 // [2][2][BM][8] fp16
   static constexpr int BAR_OFF = SC_OFF + 2 * SC_BYTES;
-  static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + 2 * A_ST + 2 + 4;
+  static constexpr int NBARS = 2 * RAW_ST + 2 * B_ST + A_ST + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM = 1024 + MISC_OFF + 64;
   static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -259,8 +259,10 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
   uint64_t* b_full = raw_empty + RAW_ST;
   uint64_t* b_empty = b_full + B_ST;
   uint64_t* a_full = b_empty + B_ST;
-  uint64_t* a_empty = a_full + A_ST;
-  uint64_t* acc_full = a_empty + A_ST;
+  // An A stage is free again when the MMAs of the stage that last used it
+  // are done, and those MMAs' commit to the token-row ring says so: the
+  // dequantising warps wait on b_empty of that stage, one commit per stage.
+  uint64_t* acc_full = a_full + A_ST;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* sc_full = acc_empty + 1;           // [2] scale blocks
   uint64_t* sc_empty = sc_full + 2;            // [2]
@@ -281,13 +283,12 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     }
     for (int s = 0; s < B_ST; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+      mbar_init(&b_empty[s], 2);          // one commit per MMA-issuing thread
     }
     for (int s = 0; s < A_ST; ++s) {
       mbar_init(&a_full[s], BM);
-      mbar_init(&a_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, 2);
     mbar_init(acc_empty, Roles<OP>::NEPI * 32);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sc_full[b], 1);
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
 
   if (warp == W_TMA) {
     // -------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+    {
       const CUtensorMap* map_slot1 = OP == 0 ? &map_q1 : &map_q0;
       const CUtensorMap* smap_slot1 = OP == 0 ? &map_s1 : &map_s0;
       const int SPB = SC_GROUPS * G / BK;     // stages per scale block (4, 8 or 16)
@@ -332,29 +333,35 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
             // groups kb * BK / G .. + 8 (x coordinate a multiple of 8)
             const int ss = gs & 1;
             if (gs >= 2 &&
-                !mbar_wait(&sc_empty[ss], ((gs >> 1) - 1) & 1, abort_flag, args.err)) {
+                !mbar_wait_warp(&sc_empty[ss], ((gs >> 1) - 1) & 1, abort_flag, args.err)) {
               stop = true;
               break;
             }
+            if (lane == 0) {
             mbar_arrive_expect_tx(&sc_full[ss], SC_BYTES);
             tma_load_2d(sSc + ss * SC_BYTES, &map_s0, kb * BK / G, U.wrow[0], &sc_full[ss]);
             tma_load_2d(sSc + ss * SC_BYTES + SC_BYTES / 2, smap_slot1, kb * BK / G, U.wrow[1],
                         &sc_full[ss]);
+            }
+            __syncwarp();
             ++gs;
           }
           if (kb % RK != 0) continue;       // this copy holds RK K stages
           const uint32_t gr = g / RK;
           const int s = gr % RAW_ST;
           if (gr >= (uint32_t)RAW_ST &&
-              !mbar_wait(&raw_empty[s], ((gr / RAW_ST) - 1) & 1, abort_flag, args.err)) {
+              !mbar_wait_warp(&raw_empty[s], ((gr / RAW_ST) - 1) & 1, abort_flag, args.err)) {
             stop = true;
             break;
           }
+          if (lane == 0) {
           mbar_arrive_expect_tx(&raw_full[s], 2 * RAW_SLOT);
           tma_load_2d(sRaw + (s * 2 + 0) * RAW_SLOT, &map_q0, kb * (BK / 2), U.wrow[0],
                       &raw_full[s]);
           tma_load_2d(sRaw + (s * 2 + 1) * RAW_SLOT, map_slot1, kb * (BK / 2), U.wrow[1],
                       &raw_full[s]);
+          }
+          __syncwarp();
         }
       }
     }
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     // -------------------------------------------------------------- token rows (B)
     // one TMA tile of 128 grouped rows per stage (rows past the unit belong
     // to other units or lie beyond S; the MMA reads only nrows of them)
-    if (lane == 0) {
+    {
       uint32_t g = 0;
       bool stop = false;
       for (int i = 0; i < my_units && !stop; ++i) {
@@ -370,25 +377,35 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % B_ST;
           if (g >= (uint32_t)B_ST &&
-              !mbar_wait(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
+              !mbar_wait_warp(&b_empty[s], ((g / B_ST) - 1) & 1, abort_flag, args.err)) {
             stop = true;
             break;
           }
+          if (lane == 0) {
           mbar_arrive_expect_tx(&b_full[s], B_BYTES);
           tma_load_2d(sB + s * B_BYTES, &map_b, kb * BK, U.p0, &b_full[s]);
+          }
+          __syncwarp();
         }
       }
     }
-  } else if (warp == W_MMA) {
+  } else if (warp == W_MMA || warp == W_MMA2) {
     // -------------------------------------------------------------- MMA issue
-    // The whole warp follows the rings; one lane, elected once, issues every
-    // MMA and commit (a commit covers the MMAs of the thread that issues it).
+    // Two warps issue the MMAs, one per slot: a thread issues one
+    // tcgen05.mma per ~64 cycles at most, which is all the time an M = 128,
+    // N = 128, K = 16 product takes, so one issuing thread alone leaves the
+    // tensor pipe idle whenever it does anything else.  Each warp follows the
+    // rings as a whole; one lane, elected once, issues its slot's MMAs and
+    // one commit per stage (a commit covers the MMAs of the thread that
+    // issues it; the rings' empty barriers count both threads' commits).
+    const int m = warp == W_MMA ? 0 : 1;
     uint32_t g = 0;
     bool stop = false;
     const bool leader = elect_one();
     for (int i = 0; i < my_units && !stop; ++i) {
       const Unit U = decode_unit<OP>(args, blockIdx.x + i * gridDim.x, FB);
       const uint32_t idesc = idesc_f32acc(BM, U.nrows, kFmtF16, 0);
+      const bool issue = leader && m < U.nslots;
       if (i > 0) {
         if (!mbar_wait_warp(acc_empty, (i - 1) & 1, abort_flag, args.err)) break;
         tc_fence_after();
@@ -401,21 +418,16 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        if (leader) {
+        if (issue) {
           const uint32_t b0 = smem_addr(sB + sb * B_BYTES);
+          const uint32_t a0 = tmem + A_COL + sa * 64 + m * 32;
 #pragma unroll
-          for (int ks = 0; ks < BK / 16; ++ks) {
-            const uint64_t bd = desc_kmajor_sw128(b0 + ks * 32);
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              if (m < U.nslots)
-                mma_f16kind_ts(tmem + m * NT, tmem + A_COL + sa * 64 + m * 32 + ks * 8, bd,
-                               idesc, (kb | ks) != 0);
-            }
-          }
-          mma_commit(&a_empty[sa]);
-          mma_commit(&b_empty[sb]);
+          for (int ks = 0; ks < BK / 16; ++ks)
+            mma_f16kind_ts(tmem + m * NT, a0 + ks * 8, desc_kmajor_sw128(b0 + ks * 32), idesc,
+                           (kb | ks) != 0);
         }
+        // frees token-row slot sb and A stage sa once both threads' MMAs are done
+        if (leader) mma_commit(&b_empty[sb]);
         __syncwarp();
       }
       if (!stop && leader) mma_commit(acc_full);
@@ -592,16 +604,16 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         // before the next TMA write into it.
         fence_proxy_async_smem();
         mbar_arrive(&raw_empty[sr]);
-        if (g >= A_ST &&
-            !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
+        if (g >= A_ST && !mbar_wait_warp(&b_empty[(g - A_ST) % B_ST], ((g - A_ST) / B_ST) & 1,
+                                         abort_flag, args.err))
           break;
         __syncwarp();       // converged before the .sync.aligned TMEM stores
         tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
         tmem_st_32x32b_x32(t_lane + A_COL + sa * 64, out0);
         tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + 32, out1);
       } else {
-        if (g >= A_ST &&
-            !mbar_wait_warp(&a_empty[sa], ((g / A_ST) - 1) & 1, abort_flag, args.err))
+        if (g >= A_ST && !mbar_wait_warp(&b_empty[(g - A_ST) % B_ST], ((g - A_ST) / B_ST) & 1,
+                                         abort_flag, args.err))
           break;
         __syncwarp();
         tc_fence_after();
