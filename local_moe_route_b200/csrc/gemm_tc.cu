@@ -26,7 +26,7 @@
 // Keeping A out of shared memory leaves shared-memory bandwidth to the B
 // tiles and the packed weights; the MMAs' own reads of B need half of it.
 //
-// Warp roles (gate/up 512 threads, down 768; persistent, one CTA per SM):
+// Warp roles (gate/up 640 threads, down 768; persistent, one CTA per SM):
 //   warp 0       TMA of packed int4 rows into a ring of 8 (down: 6) K stages
 //                of 64: one copy covers two K stages when K is a multiple of
 //                128 (a 64-byte row segment per weight row, 64-byte swizzle;
@@ -43,14 +43,14 @@
 //                token-order copy with tile::gather4 copies instead, 32 per
 //                stage, left the MMA waiting on them 64% of the time and
 //                doubled the kernel's time at T = 6144.)
-//   warps 4-11   two (down: three, warps 4-15) dequantising warpgroups taking
+//   warps 4-15   three dequantising warpgroups taking
 //                the stages round-robin; thread = weight row; fp16 pairs go to
 //                TMEM with tcgen05.st; at each scale block a thread copies its
 //                rows' 8 scales into registers and frees the ring slot.  (When
 //                K / G is not a multiple of 8 the rows' scales are loaded from
 //                global memory one block ahead instead: a thread's next
 //                release of a ring slot waits for such a load in flight.)
-//   warps 12-15  epilogue (down: warps 16-23, four per 128-feature slice):
+//   warps 16-19  epilogue (down: warps 16-23, four per 128-feature slice):
 //                TMEM -> registers -> SwiGLU or row scale -> fp16,
 //                transposed through shared memory into whole-row stores
 // TMEM (512 columns): accumulators of slot 0/1 at columns 0/160, three A
@@ -82,14 +82,15 @@ constexpr int SC_GROUPS = 8;
 constexpr int SC_BYTES = 2 * BM * SC_GROUPS * 2;   // 4 KB per block
 
 constexpr int W_TMA = 0, W_MMA = 1, W_BTMA = 2, W_MMA2 = 3, W_DQ = 4;
-// Dequantising warpgroups take the stages round-robin: two for gate/up,
-// three for down, whose units are short (K = n) and leave the MMA warp
-// waiting on dequantisation more often (measured: down 0.73 -> 0.67 ms at the
-// large shape with three, gate/up slightly slower).  Registers bound the
-// count: three groups fit at 96 registers per thread.
+// Dequantising warpgroups take the stages round-robin, three of them: with
+// the MMAs issued from two threads the MMA warps wait on dequantised A
+// stages (measured at T = 6144: gate/up 1.18 -> 1.14 ms with three groups
+// instead of two, down 0.73 -> 0.67 ms).  Registers bound the count: three
+// groups fit at 96 registers per thread (gate/up) and four epilogue warps
+// more at 80 (down).
 template <int OP>
 struct Roles {
-  static constexpr int NWG = OP == 0 ? 2 : 3;
+  static constexpr int NWG = 3;
   static constexpr int W_EPI = W_DQ + 4 * NWG;
   // epilogue warps: down has two 128-feature slices per unit and gives each
   // its own four warps, so the accumulator is read out in half the time
@@ -580,10 +581,9 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
         raw[m][0] = *reinterpret_cast<const uint4*>(rowp + 16 * (c0 ^ sw));
         raw[m][1] = *reinterpret_cast<const uint4*>(rowp + 16 * ((c0 + 1) ^ sw));
       }
-      // gate/up: both slots are dequantised into registers before this warp
-      // waits for its A stage, so a stage the MMAs release is refilled at
-      // once; down (three warpgroups at 96 registers) has no room for that
-      // and dequantises slot by slot after the wait.
+      // The slots are dequantised one after the other once the A stage is
+      // free (dequantising both into registers first, then waiting, needs
+      // more registers than three warpgroups have).
       auto dq_slot = [&](int m, uint32_t(&out)[32]) {
         const uint32_t sc_a = sc2[m][0], sc_b = sc2[m][1];
         const uint32_t words[8] = {raw[m][0].x, raw[m][0].y, raw[m][0].z, raw[m][0].w,
@@ -596,36 +596,19 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
           else dequant8(words[c], c < 4 ? sc_a : sc_b, &out[4 * c]);
         }
       };
-      if constexpr (OP == 0) {
-        uint32_t out0[32], out1[32];
-        dq_slot(0, out0);
-        dq_slot(1, out1);
-        // Release the raw stage: the fence orders the loads of its words
-        // before the next TMA write into it.
-        fence_proxy_async_smem();
-        mbar_arrive(&raw_empty[sr]);
-        if (g >= A_ST && !mbar_wait_warp(&b_empty[(g - A_ST) % B_ST], ((g - A_ST) / B_ST) & 1,
-                                         abort_flag, args.err))
-          break;
-        __syncwarp();       // converged before the .sync.aligned TMEM stores
-        tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
-        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64, out0);
-        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + 32, out1);
-      } else {
-        if (g >= A_ST && !mbar_wait_warp(&b_empty[(g - A_ST) % B_ST], ((g - A_ST) / B_ST) & 1,
-                                         abort_flag, args.err))
-          break;
-        __syncwarp();
-        tc_fence_after();
+      if (g >= A_ST && !mbar_wait_warp(&b_empty[(g - A_ST) % B_ST], ((g - A_ST) / B_ST) & 1,
+                                       abort_flag, args.err))
+        break;
+      __syncwarp();       // converged before the .sync.aligned TMEM stores
+      tc_fence_after();   // order the TMEM stores after the MMAs that released this A stage
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          uint32_t out[32];
-          dq_slot(m, out);
-          tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
-        }
-        fence_proxy_async_smem();      // the words' loads before the next TMA write
-        mbar_arrive(&raw_empty[sr]);
+      for (int m = 0; m < 2; ++m) {
+        uint32_t out[32];
+        dq_slot(m, out);
+        tmem_st_32x32b_x32(t_lane + A_COL + sa * 64 + m * 32, out);
       }
+      fence_proxy_async_smem();      // the words' loads before the next TMA write
+      mbar_arrive(&raw_empty[sr]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&a_full[sa]);
