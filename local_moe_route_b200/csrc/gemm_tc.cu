@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     moe_gemm_q4_tc_kernel(const __grid_constant__ CUtensorMap map_q0,
                           const __grid_constant__ CUtensorMap map_q1,
                           const __grid_constant__ CUtensorMap map_b,
+                          const __grid_constant__ CUtensorMap map_b128,
                           const __grid_constant__ CUtensorMap map_s0,
                           const __grid_constant__ CUtensorMap map_s1, const TcArgs args) {
   using namespace tc;
@@ -302,6 +303,7 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
     prefetch_tmap(&map_q0);
     if (OP == 0) prefetch_tmap(&map_q1);
     prefetch_tmap(&map_b);
+    prefetch_tmap(&map_b128);
     if (STMA) {
       prefetch_tmap(&map_s0);
       if (OP == 0) prefetch_tmap(&map_s1);
@@ -382,9 +384,11 @@ __global__ void __launch_bounds__(tc::Roles<OP>::THREADS, 1)
             stop = true;
             break;
           }
+          // a unit of at most 128 rows takes a 128-row tile
           if (lane == 0) {
-          mbar_arrive_expect_tx(&b_full[s], B_BYTES);
-          tma_load_2d(sB + s * B_BYTES, &map_b, kb * BK, U.p0, &b_full[s]);
+            const bool small = U.nrows <= 128;
+            mbar_arrive_expect_tx(&b_full[s], small ? 128 * BK * 2 : B_BYTES);
+            tma_load_2d(sB + s * B_BYTES, small ? &map_b128 : &map_b, kb * BK, U.p0, &b_full[s]);
           }
           __syncwarp();
         }
@@ -780,8 +784,12 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   // B rows: grouped fp16 rows [S][K] (the gathered copy of x, or h)
   CUtensorMap mb;
   const uint16_t* brows = OP == 0 ? p.a16 : p.a;
+  CUtensorMap mb128;
   if (encode_tmap_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, brows, p.K, p.S, (uint64_t)p.K * 2,
                      tc::BK, tc::NT, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS ||
+      encode_tmap_2d(&mb128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, brows, p.K, p.S, (uint64_t)p.K * 2,
+                     tc::BK, 128, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (OP == 0 &&
@@ -838,7 +846,7 @@ static cudaError_t launch_tc_impl(const GemmProblem& p, const Schedule& sch, cud
   const long max_units = (long)max_tiles(p.S, p.E) * FB;
   const int grid = (int)(max_units < num_sms ? max_units : num_sms);
   moe_gemm_q4_tc_kernel<OP, ILV, STMA><<<grid, tc::Roles<OP>::THREADS, tc::Lay<OP, RK>::SMEM, s>>>(
-      m0, m1, mb, ms0, ms1, a);
+      m0, m1, mb, mb128, ms0, ms1, a);
   return cudaGetLastError();
 }
 
