@@ -8,7 +8,8 @@
 // together), so the step is bound by HBM bandwidth over those bytes plus the
 // fixed cost between the weight streams.  Here that fixed cost is one
 // launch: the CTAs stay resident (cooperative launch, two per SM) and pass
-// through five phases separated by grid-wide barriers with bounded waits:
+// through five phases, separated by grid-wide barriers or per-expert
+// counters with bounded waits:
 //
 //   P0  router partial logits (items of 128 rows of W_r x 64 experts);
 //       every CTA also converts x of all tokens to fp16 in shared memory;
@@ -23,9 +24,12 @@
 //   P2  gate/up + SwiGLU: units of 16 weight rows of one expert, K split
 //       over the 8 consumer warps, both matrices streamed by TMA through a
 //       3-deep ring, B operand = x from shared memory; h to global (fp16);
-//   --- grid barrier
+//       each stored unit adds one to its expert's counter;
 //   P3  down: units of 64 rows of one expert (4 row groups x 2 K halves),
-//       each stage carries the expert's h rows; output rows to global (fp32);
+//       each stage carries the expert's h rows, loaded once the expert's
+//       counter shows all of its gate/up units (a CTA starts its down units
+//       while others still finish gate/up ones); output rows to global
+//       (fp32);
 //   --- grid barrier
 //   P4  combine: y_t = sum_j w_tj * row_(t,j), fp32 in slot order, bf16.
 //
@@ -112,8 +116,9 @@ struct FusedArgs {
   float* logits;             // [T][E]
   uint16_t* h;               // [T*k][n] fp16, features interleaved within 8
   float* rows;               // [T*k][d] fp32
-  unsigned* sync;            // [8] zeroed before the launch: [0] barrier arrivals,
-                             // [2] abort, [4] / [5] gate-up / down unit counters
+  unsigned* sync;            // zeroed before the launch: [0] barrier arrivals,
+                             // [2] abort, [4] / [5] gate-up / down unit counters,
+                             // [64 + i] gate/up units of active expert i done
   unsigned* err;
   int T, d, E, k, n, G;
 };
@@ -134,6 +139,34 @@ __device__ __forceinline__ bool df_sync_grid(unsigned* sync, int b, unsigned* er
   // barrier and after its own earlier generic accesses of shared memory
   asm volatile("fence.proxy.async;" ::: "memory");
   return ok;
+}
+
+// One thread: waits until *cnt reaches `target` (acquire), then orders its
+// later TMA reads of global memory after it.  Gives up after kWaitLimitNs or
+// when a CTA has raised the grid-wide abort, and then raises this CTA's
+// abort; a time-out also records kErrTimeout and raises the grid-wide one.
+__device__ __forceinline__ bool df_wait_count(const unsigned* cnt, unsigned target, unsigned* sync,
+                                              unsigned* err, volatile int* cta_abort) {
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
+    unsigned v, ab;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (v >= target) {
+      asm volatile("fence.proxy.async;" ::: "memory");
+      return true;
+    }
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(sync + 2) : "memory");
+    if (ab || *cta_abort) {
+      *cta_abort = 1;
+      return false;
+    }
+    if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) break;
+    __nanosleep(64);
+  }
+  atomicOr(err, kErrTimeout);
+  *cta_abort = 1;
+  atomicExch(&sync[2], 1u);
+  return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -742,6 +775,12 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             a.h[(size_t)(prow + col) * a.n + df_ilv(fb * P2_ROWS + r)] = f16_bits(hv);
           }
         }
+        // the unit's h values, then one more finished unit of the expert:
+        // the down phase of any CTA may read the expert's h once all of its
+        // gate/up units are counted
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(&a.sync[64 + u / FB2], 1u);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red_empty[b]);
@@ -750,7 +789,11 @@ __global__ void __launch_bounds__(df::THREADS, 2)
     }
     rc = rr;
   }
-  ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
+  // No grid barrier here: a CTA goes on to down units as soon as its own
+  // gate/up work is done, and its producer waits, per unit, until every
+  // gate/up unit of that unit's expert has stored its h (a counter per
+  // active expert) before it loads h; the down weights of the stage are
+  // already on their way by then.
 
   // ---- P3: down, units (expert, 64 rows): 4 row groups x 2 K halves
   const int FB3 = a.d / P3_ROWS, KS3 = a.n / P3_KST;
@@ -781,8 +824,17 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           mbar_arrive_expect_tx(&full[s], P3_ROWS * (P3_KST / 2) + MAXT * P3_KST * 2 +
                                               P3_ROWS * (a.n / G) * 2);
           tma_load_2d(sl, &map_wd, kc * (P3_KST / 2), wrow, &full[s]);
-          tma_load_2d(sl + P3_H, &map_h, kc * P3_KST, prow, &full[s]);
           tma_load_2d(sl + P3_SC, &map_sd, 0, wrow, &full[s]);     // the unit's scale rows
+          const bool ready =
+              kc != 0 || df_wait_count(&a.sync[64 + u / FB3], (unsigned)FB2, a.sync, a.err,
+                                       abort_flag);
+          // loaded either way, so the stage's copies all complete; after a
+          // wait that gave up the CTA's roles are already winding down
+          tma_load_2d(sl + P3_H, &map_h, kc * P3_KST, prow, &full[s]);
+          if (!ready) {
+            stop = true;
+            break;
+          }
         }
         if (stop || last) break;
         u = nx;
@@ -869,7 +921,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       if (u < 0) break;
     }
   }
-  ok = df_sync_grid(a.sync, 3, a.err, flag, abort_flag) && ok;
+  ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
 
   // ---- P4: combine, fp32 in slot order j = 0 .. k-1, one rounding to bf16
   if (ok) {
@@ -929,7 +981,7 @@ size_t decode_fused_scratch(int T, int d, int E, int k, int n) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t S = (size_t)T * k;
   return up((size_t)(d / df::P0_RS) * T * E * 4) + up((size_t)T * E * 4) + up(S * n * 2) +
-         up(S * d * 4) + 256;
+         up(S * d * 4) + 256 + 4 * df::MAXS;
 }
 
 template <int G>
@@ -1019,7 +1071,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, const uint16_t* w_router, con
                      (uint64_t)(n / G) * 2, n / G, P3_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.sync, 0, 32, s);   // barrier words, unit counters
+  // barrier words, unit counters and the per-expert counts of finished units
+  cudaError_t e = cudaMemsetAsync(a.sync, 0, 256 + 4 * (size_t)T * k, s);
   if (e != cudaSuccess) return e;
   const int smem = Smem::of(T, d).total + 1024;
   if (G == 32) return launch_fused_g<32>(maps, a, smem, s);
