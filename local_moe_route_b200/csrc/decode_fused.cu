@@ -29,9 +29,10 @@
 //       each stage carries the expert's h rows, loaded once the expert's
 //       counter shows all of its gate/up units (a CTA starts its down units
 //       while others still finish gate/up ones); output rows to global
-//       (fp32);
-//   --- grid barrier
-//   P4  combine: y_t = sum_j w_tj * row_(t,j), fp32 in slot order, bf16.
+//       (fp32); each stored unit adds one to a count of finished units;
+//   P4  combine: y_t = sum_j w_tj * row_(t,j), fp32 in slot order, bf16, in
+//       the CTAs that have combine items, once the count shows every down
+//       unit (the other CTAs end after P3).
 //
 // Warp roles in P2 and P3: one producer warp (TMA), eight consumer warps
 // (matrix products) and one reducer warp.  The units are handed out
@@ -118,6 +119,7 @@ struct FusedArgs {
   float* rows;               // [T*k][d] fp32
   unsigned* sync;            // zeroed before the launch: [0] barrier arrivals,
                              // [2] abort, [4] / [5] gate-up / down unit counters,
+                             // [6] down units done,
                              // [64 + i] gate/up units of active expert i done
   unsigned* err;
   int T, d, E, k, n, G;
@@ -914,6 +916,10 @@ __global__ void __launch_bounds__(df::THREADS, 2)
             a.rows[(size_t)(prow + col) * a.d + fb * P3_ROWS + row] = v;
           }
         }
+        // the unit's rows, then one more finished down unit
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(&a.sync[6], 1u);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red_empty[b]);
@@ -921,11 +927,17 @@ __global__ void __launch_bounds__(df::THREADS, 2)
       if (u < 0) break;
     }
   }
-  ok = df_sync_grid(a.sync, 2, a.err, flag, abort_flag) && ok;
-
-  // ---- P4: combine, fp32 in slot order j = 0 .. k-1, one rounding to bf16
+  // ---- P4: combine, fp32 in slot order j = 0 .. k-1, one rounding to bf16.
+  // Only the CTAs with combine items take part; they wait for the count of
+  // finished down units instead of a grid barrier, and the others are done.
+  const int cpr = a.d / 8;
+  if ((int)(blockIdx.x * blockDim.x) >= a.T * cpr) return;
+  __syncthreads();
+  if (threadIdx.x == 0)
+    *flag = ok && df_wait_count(&a.sync[6], (unsigned)units3, a.sync, a.err, abort_flag) ? 1 : 0;
+  __syncthreads();
+  ok = *flag != 0;
   if (ok) {
-    const int cpr = a.d / 8;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.T * cpr; i += gridDim.x * blockDim.x) {
       const int tk = i / cpr, f0 = (i % cpr) * 8;
       float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
