@@ -313,16 +313,28 @@ __global__ void __launch_bounds__(128)
   if (t >= T) return;
   uint32_t key[VPL];
   uint32_t taken = 0;                         // entries already picked
+  // the lane's VPL logits of split sp are loaded together (one round trip
+  // per split, not one per logit), and the splits added in order
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  for (int sp = 0; sp < ksplit; ++sp) {
+    const float* src = partial + ((size_t)sp * T + t) * E + lane;
+    float v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) v[i] = lane + 32 * i < E ? src[32 * i] : 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc[i] += v[i];
+  }
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
     key[i] = 0u;
     if (e < E) {
-      float acc = 0.f;
-      for (int sp = 0; sp < ksplit; ++sp) acc += partial[((size_t)sp * T + t) * E + e];
-      if (bias) acc += bias[e];
-      if (logits_out) logits_out[(size_t)t * E + e] = acc;
-      key[i] = logit_key(acc);
+      float a = acc[i];
+      if (bias) a += bias[e];
+      if (logits_out) logits_out[(size_t)t * E + e] = a;
+      key[i] = logit_key(a);
     }
   }
   uint32_t my_key = 0, top = 0;
