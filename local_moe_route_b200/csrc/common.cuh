@@ -156,35 +156,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Same, with an L2 eviction-priority policy (from l2_policy_*) for the bytes read.
-__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int32_t x,
-                                                 int32_t y, uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-
-// Four rows of a 2-D tensor (the map's box is one row high) into four
-// consecutive box-sized rows of shared memory: columns x.. of rows r[0..3].
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int32_t x,
-                                            const int (&r)[4], uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
-      "r"(smem_addr(bar))
-      : "memory");
-}
-
-// L2 policies: data read once (streamed weights) leaves L2 first.
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
 // Before a thread releases a shared-memory slot that TMA (the async proxy)
 // will overwrite: orders this thread's earlier generic reads of the slot
 // before those writes.  Without it a load whose result is consumed only
