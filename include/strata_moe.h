@@ -297,7 +297,7 @@ STRATA_API strata_status_t strata_moe_device_status(strata_stream_t stream);
  * wait in the kernels above is bounded in the same way (about one second),
  * after which the kernel records a time-out in the device check word,
  * releases what it holds and returns instead of spinning forever.
- *   out      device int32[8] (16-byte aligned), written by the kernels:
+ *   out      device int32[10] (16-byte aligned), written by the kernels:
  *            out[0..3]  1 if wait w completed, 0 if it gave up (an mbarrier
  *                       that nothing arrives on; warp 0 waits alone, warps
  *                       1..3 wait as whole warps and see warp 0's abort;
@@ -307,7 +307,11 @@ STRATA_API strata_status_t strata_moe_device_status(strata_stream_t stream);
  *            out[6]     1 if a two-CTA grid barrier that one CTA never
  *                       reaches completed, 0 if it gave up
  *            out[7]     nanoseconds that barrier waited
- *   sync_ws  device scratch of 16 bytes (16-byte aligned), overwritten
+ *            out[8]     1 if a wait for a count of finished work that
+ *                       nothing raises (the form the fused decode kernel
+ *                       uses between its phases) completed, 0 if it gave up
+ *            out[9]     nanoseconds that wait took
+ *   sync_ws  device scratch of 32 bytes (16-byte aligned), overwritten
  * Both kernels take about one second each.  Afterwards
  * strata_moe_device_status() reports STRATA_ERR_DEVICE_CHECK (and clears it);
  * the device stays usable. */

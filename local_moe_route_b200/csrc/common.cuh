@@ -144,6 +144,35 @@ __device__ __forceinline__ bool grid_barrier_wait(unsigned* sync, int b, unsigne
 }
 
 
+// One thread: waits until *cnt reaches `target` (acquire), then orders its
+// later TMA reads of global memory after it.  Gives up after kWaitLimitNs or
+// when *grid_abort is raised, and then raises the CTA's abort flag; a
+// time-out also records kErrTimeout and raises *grid_abort.
+__device__ __forceinline__ bool counter_wait(const unsigned* cnt, unsigned target,
+                                             unsigned* grid_abort, unsigned* err,
+                                             volatile int* cta_abort) {
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
+    unsigned v, ab;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (v >= target) {
+      asm volatile("fence.proxy.async;" ::: "memory");
+      return true;
+    }
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(grid_abort) : "memory");
+    if (ab || *cta_abort) {
+      *cta_abort = 1;
+      return false;
+    }
+    if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) break;
+    __nanosleep(64);
+  }
+  atomicOr(err, kErrTimeout);
+  *cta_abort = 1;
+  atomicExch(grid_abort, 1u);
+  return false;
+}
+
 // ---------------------------------------------------------------------------
 // TMA copies
 // 2-D TMA tile load global -> shared, completion counted on `bar` in bytes.

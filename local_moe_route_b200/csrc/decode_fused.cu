@@ -143,34 +143,6 @@ __device__ __forceinline__ bool df_sync_grid(unsigned* sync, int b, unsigned* er
   return ok;
 }
 
-// One thread: waits until *cnt reaches `target` (acquire), then orders its
-// later TMA reads of global memory after it.  Gives up after kWaitLimitNs or
-// when a CTA has raised the grid-wide abort, and then raises this CTA's
-// abort; a time-out also records kErrTimeout and raises the grid-wide one.
-__device__ __forceinline__ bool df_wait_count(const unsigned* cnt, unsigned target, unsigned* sync,
-                                              unsigned* err, volatile int* cta_abort) {
-  const unsigned long long t0 = global_ns();
-  for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
-    unsigned v, ab;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-    if (v >= target) {
-      asm volatile("fence.proxy.async;" ::: "memory");
-      return true;
-    }
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(sync + 2) : "memory");
-    if (ab || *cta_abort) {
-      *cta_abort = 1;
-      return false;
-    }
-    if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) break;
-    __nanosleep(64);
-  }
-  atomicOr(err, kErrTimeout);
-  *cta_abort = 1;
-  atomicExch(&sync[2], 1u);
-  return false;
-}
-
 // ---------------------------------------------------------------------------
 // P0: partial router logits.  Item = (128 rows of W_r, 64 experts): thread
 // (row group rr = th / 8 of 32, 16-byte chunk c = th % 8 of 8 experts) loads
@@ -828,8 +800,8 @@ __global__ void __launch_bounds__(df::THREADS, 2)
           tma_load_2d(sl, &map_wd, kc * (P3_KST / 2), wrow, &full[s]);
           tma_load_2d(sl + P3_SC, &map_sd, 0, wrow, &full[s]);     // the unit's scale rows
           const bool ready =
-              kc != 0 || df_wait_count(&a.sync[64 + u / FB3], (unsigned)FB2, a.sync, a.err,
-                                       abort_flag);
+              kc != 0 || counter_wait(&a.sync[64 + u / FB3], (unsigned)FB2, &a.sync[2], a.err,
+                                      abort_flag);
           // loaded either way, so the stage's copies all complete; after a
           // wait that gave up the CTA's roles are already winding down
           tma_load_2d(sl + P3_H, &map_h, kc * P3_KST, prow, &full[s]);
@@ -934,7 +906,7 @@ __global__ void __launch_bounds__(df::THREADS, 2)
   if ((int)(blockIdx.x * blockDim.x) >= a.T * cpr) return;
   __syncthreads();
   if (threadIdx.x == 0)
-    *flag = ok && df_wait_count(&a.sync[6], (unsigned)units3, a.sync, a.err, abort_flag) ? 1 : 0;
+    *flag = ok && counter_wait(&a.sync[6], (unsigned)units3, &a.sync[2], a.err, abort_flag) ? 1 : 0;
   __syncthreads();
   ok = *flag != 0;
   if (ok) {

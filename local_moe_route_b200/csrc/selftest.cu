@@ -2,8 +2,9 @@
 // purpose, so that the give-up path (record kErrTimeout, raise the abort
 // flag, release what the kernel holds, return) is exercised on the device.
 // Each wait here is on a condition that nothing ever satisfies: an mbarrier
-// that no thread or copy arrives on, and a grid barrier that one CTA never
-// reaches.  Nothing traps and nothing waits without a limit.
+// that no thread or copy arrives on, a grid barrier that one CTA never
+// reaches, and a counter of finished work that nothing raises.  Nothing
+// traps and nothing waits without a limit.
 #include "../../include/strata_moe.h"
 #include "common.cuh"
 #include "internal.h"
@@ -52,15 +53,27 @@ __global__ void __launch_bounds__(128, 1) selftest_mbar_kernel(int32_t* out, uns
   }
 }
 
-// Two CTAs (cooperative launch); CTA 1 never arrives at the grid barrier.
+// Two CTAs (cooperative launch); CTA 1 never arrives at the grid barrier
+// (sync[0], abort word sync[2]).  Meanwhile CTA 1 waits for a counter that
+// nothing raises (sync[4], abort word sync[6]).
 //   out[6] 1 if CTA 0's barrier completed, 0 if it gave up
 //   out[7] nanoseconds CTA 0 waited
+//   out[8] 1 if CTA 1's counter wait completed, 0 if it gave up
+//   out[9] nanoseconds CTA 1 waited
 __global__ void selftest_grid_kernel(int32_t* out, unsigned* sync, unsigned* err) {
-  if (blockIdx.x != 0 || threadIdx.x != 0) return;
+  __shared__ int cta_abort;
+  if (threadIdx.x != 0) return;
   const unsigned long long t0 = global_ns();
-  const bool ok = grid_barrier_wait(sync, 0, err);
-  out[7] = (int32_t)min(global_ns() - t0, 2000000000ull);
-  out[6] = ok ? 1 : 0;
+  if (blockIdx.x == 0) {
+    const bool ok = grid_barrier_wait(sync, 0, err);
+    out[7] = (int32_t)min(global_ns() - t0, 2000000000ull);
+    out[6] = ok ? 1 : 0;
+  } else {
+    cta_abort = 0;
+    const bool ok = counter_wait(&sync[4], 1u, &sync[6], err, &cta_abort);
+    out[9] = (int32_t)min(global_ns() - t0, 2000000000ull);
+    out[8] = ok ? 1 : 0;
+  }
 }
 
 unsigned* check_word();
@@ -79,8 +92,8 @@ extern "C" strata_status_t strata_moe_selftest_wait(int32_t* out, void* sync_ws,
   if (!err) return STRATA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   unsigned* sync = static_cast<unsigned*>(sync_ws);
-  if (cudaMemsetAsync(out, 0, 8 * sizeof(int32_t), s) != cudaSuccess ||
-      cudaMemsetAsync(sync, 0, 16, s) != cudaSuccess)
+  if (cudaMemsetAsync(out, 0, 10 * sizeof(int32_t), s) != cudaSuccess ||
+      cudaMemsetAsync(sync, 0, 32, s) != cudaSuccess)
     return STRATA_ERR_CUDA;
   selftest_mbar_kernel<<<1, 128, 0, s>>>(out, err);
   if (cudaGetLastError() != cudaSuccess) return STRATA_ERR_CUDA;

@@ -527,11 +527,12 @@ def test_bad_offsets_are_reported_not_used(dev):
 
 def test_bounded_waits_give_up_and_leave_the_device_usable(dev):
     """Waits on conditions nothing satisfies (an mbarrier no thread or copy
-    arrives on, a grid barrier one CTA never reaches) give up after their
-    limit: the kernels return, the time-out is reported, tensor memory held
-    during the wait is released, and the next forward is correct."""
-    out = torch.full((8,), -1, dtype=torch.int32, device=dev)
-    sync = torch.zeros(16, dtype=torch.uint8, device=dev)
+    arrives on, a grid barrier one CTA never reaches, a count of finished
+    work nothing raises) give up after their limit: the kernels return, the
+    time-out is reported, tensor memory held during the wait is released,
+    and the next forward is correct."""
+    out = torch.full((10,), -1, dtype=torch.int32, device=dev)
+    sync = torch.zeros(32, dtype=torch.uint8, device=dev)
     assert sm.strata_moe_selftest_wait(out, sync) == sm.STRATA_OK
     torch.cuda.synchronize()
     o = out.cpu().tolist()
@@ -539,6 +540,7 @@ def test_bounded_waits_give_up_and_leave_the_device_usable(dev):
     assert 0.9e9 <= o[4] <= 1.9e9, o           # after about the one-second limit
     assert o[5] == 1, o                        # tensor memory released
     assert o[6] == 0 and 0.9e9 <= o[7] <= 1.9e9, o
+    assert o[8] == 0 and 0.9e9 <= o[9] <= 1.9e9, o
     assert sm.strata_moe_device_status() == sm.STRATA_ERR_DEVICE_CHECK
     assert sm.strata_moe_device_status() == sm.STRATA_OK
     L = Layer.custom(dev, T=40, d=256, E=8, k=2, n=128, group=64, seed=58)
