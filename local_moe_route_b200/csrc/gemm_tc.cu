@@ -35,8 +35,8 @@
 //                row) every 8 G / 64 stages into a two-deep ring
 //   warps 1, 3   tcgen05.mma issue, one thread per slot
 //   warp 2       token rows into a 5-deep (down: 4-deep) ring, one TMA tile
-//                of 160 rows per stage: the down projection reads h, whose
-//                rows are already
+//                of 160 rows per stage (128 for units of at most 128 rows):
+//                the down projection reads h, whose rows are already
 //                grouped by expert; for gate/up a pre-pass writes the fp16 rows
 //                of x in grouped order (x[sorted_token[p]]), so both operands
 //                of every stage arrive by TMA.  (Gathering the rows from a
