@@ -20,8 +20,9 @@ At N = 1 the line also carries
     (both rooflines) and the whole 34,000-token skewed prompt as six chunks
     (tokens/s = 34,000 / sum of chunk times, per-chunk expert load);
   * `sustained`: the headline forward run back to back for --sustain-s
-    seconds (default 60) with nvidia-smi sampled every 200 ms: the rate, the
-    median SM clock, time x clock, and step times binned by clock.
+    seconds (default 60) with the clocks sampled (NVML every 5 ms, else
+    nvidia-smi every 200 ms): the rate, the median SM clock, time x clock,
+    and step times binned by clock.
 
 --impl reference times the fp64 CPU oracle on a bounded token sample of the
 same workload on the host cores (rank 0 only).
@@ -64,19 +65,35 @@ def log(*a):
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi every 200 ms while a timed region runs; every line
-    is kept with the host time it arrived."""
+    """Samples the SM clock, power and throttle reasons while a timed region
+    runs: through NVML every 5 ms when it is available (a 100 ms timed
+    region then has about 20 samples), else nvidia-smi every 200 ms.  Every
+    sample is kept as an nvidia-smi CSV line (FIELDS order) with the host
+    time it was taken."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    NVML_PERIOD_S = 0.005
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.nvml = None
         self.lines = []          # (host time, csv line)
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.nvml = (pynvml, handle)
+            self.stop_event = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
@@ -87,11 +104,43 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    @classmethod
+    def nvml_line(cls, nv, handle, index):
+        """One sample from NVML in the CSV form nvidia-smi prints for FIELDS."""
+        sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        try:
+            pw = "%.2f" % (nv.nvmlDeviceGetPowerUsage(handle) / 1000.0)
+        except Exception:
+            pw = "[N/A]"
+        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        flags = ["Active" if mask & b else "Not Active" for b in bits]
+        return ", ".join([str(index), str(sm), str(mx), pw, "0x%016x" % mask] + flags)
+
+    def _poll(self):
+        nv, handle = self.nvml
+        while not self.stop_event.is_set():
+            try:
+                self.lines.append((time.time(), self.nvml_line(nv, handle, self.index)))
+            except Exception:
+                return
+            time.sleep(self.NVML_PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
 
     def stop(self):
+        if self.nvml is not None:
+            self.stop_event.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
+            return self.summarise([ln for _, ln in self.lines])
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -739,8 +788,8 @@ def run_secondary_attention(sm, dev, aw, args):
 
 # --------------------------------------------------------------------------- sustained
 def run_sustained(R, seconds, dev, tf_burst, tf_sus, peak_kind):
-    """The headline forward back to back for `seconds`, nvidia-smi sampled
-    every 200 ms.  Events every `block` steps give the step time over the run;
+    """The headline forward back to back for `seconds`, clocks sampled as in
+    ClockSampler.  Events every `block` steps give the step time over the run;
     each clock sample is paired with the block running when it was taken."""
     import torch
     stream = torch.cuda.current_stream()

@@ -99,3 +99,37 @@ def test_clock_line_parse_keeps_power_and_reasons():
     sm, mx, pw, reasons = bench.ClockSampler.parse(_line(1800, reasons=act))
     assert (sm, mx, pw, reasons) == (1800.0, 1965.0, 812.5, {"sw_power_cap"})
     assert bench.ClockSampler.parse("garbled") is None
+
+
+class _FakeNvml:
+    """Stands in for pynvml: fixed clocks, 812.5 W, and the power-cap reason."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+
+    def __init__(self, sm=1800, mask=0x4):
+        self.sm, self.mask = sm, mask
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.sm
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 812500
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.mask
+
+
+def test_nvml_sample_reads_back_like_an_nvidia_smi_line():
+    line = bench.ClockSampler.nvml_line(_FakeNvml(), None, 0)
+    assert bench.ClockSampler.parse(line) == (1800.0, 1965.0, 812.5, {"sw_power_cap"})
+    hot = bench.ClockSampler.nvml_line(_FakeNvml(sm=1500, mask=0x8 | 0x40), None, 0)
+    assert bench.ClockSampler.parse(hot)[3] == {"hw_slowdown", "hw_thermal_slowdown"}
+    c = bench.ClockSampler.summarise([line, line, hot])
+    assert c["samples"] == 3 and c["sm_mhz"] == 1800.0
+    assert c["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
